@@ -1,0 +1,187 @@
+"""CPU oracle for the quantized gated delta-rule decode step (ctypes wrapper).
+
+TEST INFRASTRUCTURE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA library: the arithmetic lives in ``stq_oracle.c`` (plain C,
+fp64 continuous part, fp32 quantisation decision), compiled here with gcc.
+
+Every function follows the page "STEPQuant: When and Where Errors Matter in
+Delta-Rule Recurrent State Quantization" (see the header of stq_oracle.c for
+the section-by-section citations and the readings taken where it is silent).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "stq_oracle.c")
+_LIB = os.path.join(_HERE, "libstq_oracle.so")
+CFLAGS = ["-O2", "-fno-tree-vectorize", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+          "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+OK, NONFINITE, BADARG = 0, 1, 2
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile stq_oracle.c into libstq_oracle.so (if missing or stale)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = C.CDLL(_LIB)
+        P = C.c_void_p
+        L.orc_page_bytes.restype = C.c_size_t
+        L.orc_page_bytes.argtypes = [C.c_int, C.c_int, P]
+        L.orc_get_code.restype = C.c_int32
+        L.orc_get_code.argtypes = [P, C.c_int, C.c_int]
+        L.orc_put_code.restype = None
+        L.orc_put_code.argtypes = [P, C.c_int, C.c_int, C.c_int32]
+        L.orc_quantize_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P, P]
+        L.orc_dequantize_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P]
+        L.orc_step_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P, P, P, P, C.c_float, P, P, P]
+        L.orc_step_unit_f64.argtypes = [C.c_int, C.c_int, P, P, P, P, C.c_float, P, P]
+        L.orc_step_many.argtypes = [C.c_int, C.c_int, C.c_int, P, P, P, P, P, P, P, P, P, P, P,
+                                    P, P, P, C.c_int]
+        L.orc_default_threads.restype = C.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _u8(a):
+    return np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def page_bytes(bits, dv: int | None = None) -> int:
+    bits = _u8(bits)
+    dv = len(bits) if dv is None else dv
+    return int(lib().orc_page_bytes(len(bits), dv, _p(bits)))
+
+
+def row_offsets(bits, dv: int | None = None) -> np.ndarray:
+    """Byte offset of every packed row inside a page (scales come first)."""
+    bits = np.asarray(bits, dtype=np.int64)
+    dv = len(bits) if dv is None else dv
+    sizes = dv * bits // 8
+    return 4 * len(bits) + np.concatenate([[0], np.cumsum(sizes)[:-1]])
+
+
+def get_code(row: np.ndarray, b: int, j: int) -> int:
+    row = _u8(row)
+    return int(lib().orc_get_code(_p(row), b, j))
+
+
+def put_code(row: np.ndarray, b: int, j: int, z: int) -> None:
+    assert row.dtype == np.uint8 and row.flags.c_contiguous
+    lib().orc_put_code(_p(row), b, j, int(z))
+
+
+def quantize_unit(bits, r, c, S, *, with_quot: bool = False):
+    """fp32 state [dk, dv] -> packed page (uint8).  Optionally the fp32
+    quotients mu / s the codes were rounded from."""
+    bits, r, c, S = _u8(bits), _f32(r), _f32(c), _f32(S)
+    dk, dv = S.shape
+    page = np.zeros(page_bytes(bits, dv), np.uint8)
+    quot = np.zeros((dk, dv), np.float32) if with_quot else None
+    st = lib().orc_quantize_unit(dk, dv, _p(bits), _p(r), _p(c), _p(S), _p(page), _p(quot))
+    if st == BADARG:
+        raise ValueError("bad bit widths")
+    return (page, quot, st) if with_quot else page
+
+
+def dequantize_unit(bits, r, c, page, dv: int | None = None) -> np.ndarray:
+    bits, r, c, page = _u8(bits), _f32(r), _f32(c), _u8(page)
+    dk = len(bits)
+    dv = dk if dv is None else dv
+    S = np.zeros((dk, dv), np.float32)
+    st = lib().orc_dequantize_unit(dk, dv, _p(bits), _p(r), _p(c), _p(page), _p(S))
+    if st == BADARG:
+        raise ValueError("bad bit widths")
+    return S
+
+
+def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None):
+    """One quantized decode step of one unit.
+
+    Returns (page_out uint8, y float64 [dv], quot float32 [dk, dv], status)."""
+    bits, r, c, page_in = _u8(bits), _f32(r), _f32(c), _u8(page_in)
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
+    dk = len(bits)
+    dv = len(v) if dv is None else dv
+    if g.size == 1:
+        g = np.full(dk, g.reshape(()), np.float32)
+    page_out = np.zeros(page_bytes(bits, dv), np.uint8)
+    y = np.zeros(dv, np.float64)
+    quot = np.zeros((dk, dv), np.float32)
+    st = lib().orc_step_unit(dk, dv, _p(bits), _p(r), _p(c), _p(page_in), _p(page_out), _p(q),
+                             _p(k), _p(v), float(beta), _p(g), _p(y), _p(quot))
+    if st == BADARG:
+        raise ValueError("bad bit widths")
+    return page_out, y, quot, st
+
+
+def step_unit_f64(S, q, k, v, beta, g):
+    """Unquantized recurrence in fp64.  Returns (S_new float64, y float64)."""
+    S = np.array(S, dtype=np.float64, order="C", copy=True)
+    q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
+    dk, dv = S.shape
+    if g.size == 1:
+        g = np.full(dk, g.reshape(()), np.float32)
+    y = np.zeros(dv, np.float64)
+    lib().orc_step_unit_f64(dk, dv, _p(S), _p(q), _p(k), _p(v), float(beta), _p(g), _p(y))
+    return S, y
+
+
+def step_many(head, bits_table, r_table, c_table, pages_in, off_in, off_out, out_size,
+              q, k, v, beta, g, nthreads: int = 0):
+    """Many units (OpenMP over units).  Tables are per head: bits [H, dk],
+    r [H, dk], c [H, dv].  Returns (pages_out uint8, y float64 [n, dv], bad)."""
+    head = np.ascontiguousarray(head, np.int32)
+    bits_table, r_table, c_table = _u8(bits_table), _f32(r_table), _f32(c_table)
+    pages_in = _u8(pages_in)
+    off_in = np.ascontiguousarray(off_in, np.int64)
+    off_out = np.ascontiguousarray(off_out, np.int64)
+    q, k, v, beta, g = _f32(q), _f32(k), _f32(v), _f32(beta), _f32(g)
+    n = len(head)
+    dk = bits_table.shape[1]
+    dv = c_table.shape[1]
+    pages_out = np.zeros(out_size, np.uint8)
+    y = np.zeros((n, dv), np.float64)
+    bad = lib().orc_step_many(n, dk, dv, _p(head), _p(bits_table), _p(r_table), _p(c_table),
+                              _p(pages_in), _p(off_in), _p(pages_out), _p(off_out), _p(q), _p(k),
+                              _p(v), _p(beta), _p(g), _p(y), int(nthreads))
+    return pages_out, y, int(bad)
+
+
+def default_threads() -> int:
+    return int(lib().orc_default_threads())
+
+
+def near_tie(quot: np.ndarray, rel: float = 1e-4) -> np.ndarray:
+    """Elements whose quotient lies within rel * |x| of a half-integer."""
+    x = np.asarray(quot, np.float64)
+    frac = np.abs(x - np.floor(x) - 0.5)
+    return frac <= rel * np.maximum(np.abs(x), 1.0)

@@ -1,0 +1,317 @@
+/*
+ * stq_oracle.c -- CPU oracle for the quantized gated delta-rule decode step.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark may load this library.  The product path
+ * (the CUDA library and its Python binding) never calls it, and the two
+ * share no code: this file has its own packer, unpacker, quantizer and
+ * recurrence, written from the method's definition, deliberately plain and
+ * slow (bit-by-bit packing, scalar loops, no blocking, no reordering).
+ *
+ * Source of every formula: the page "STEPQuant: When and Where Errors Matter
+ * in Delta-Rule Recurrent State Quantization" (paper.rainbus.top/paper/
+ * 2609.38169), cited below by its section names:
+ *   [bg-state]  background, "linear attention and recurrent state":
+ *               y_t = S_t^T q_t, S in R^{dk x dv}.
+ *   [bg-delta]  background, "gated delta rule":
+ *               S_t = (I - b_t k_t k_t^T) D_t S_{t-1} + b_t k_t v_t^T,
+ *               D_t = alpha_t I (GDN) or a per-channel diagonal (KDA).
+ *   [bg-quant]  background, "PTQ and symmetric uniform quantisation":
+ *               Q_{b,s}(x) = s clip(round(x / s), -q_b, q_b), q_b = 2^(b-1) - 1.
+ *   [bg-smooth] background, "smoothing": absmax quantisation, row factor r_i,
+ *               column factor c_j.
+ *   [core]      core method: reconstruction  X^_ij = r_i c_j z_ij.
+ *   [steps]     method steps, online decode (the paper's Table C2):
+ *               step 1 reconstruct S^_{t-1} from integer codes and scales;
+ *               step 2 X_t = D_t S^ + b_t k_t (v_t^T - k_t^T D_t S^);
+ *               step 3 emit y_t = X_t^T q_t before requantisation;
+ *               steps 4-6 scale, quantise, pack the codes and scales back.
+ *
+ * Readings taken where the page is silent (each listed in the design notes):
+ *   - one quantisation group per key row: s_i = a_i / q_b with
+ *     a_i = max_j |X_ij / (r_i c_j)| (absmax; the row factor and column
+ *     factor are frozen per-head tables);
+ *   - round() is IEEE round-half-to-even; the code -2^(b-1) is never made;
+ *   - scales are stored as fp32;
+ *   - the continuous part (reconstruction, decay, retrieval, write,
+ *     readout) is computed in fp64; the quantisation decision is taken in
+ *     fp32 on the fp32-rounded value mu_ij = fl32(X_ij / (r_i c_j)), with
+ *     IEEE fp32 division for s_i = a_i / q_b and for mu_ij / s_i;
+ *   - an all-zero row has s_i = 0 and all codes 0.
+ *
+ * Packed page of one (request, slot, head) unit, dk rows of dv codes:
+ *   bytes [0, 4 dk)        fp32 scales s_0 .. s_{dk-1} (little-endian)
+ *   then row i = 0..dk-1   dv codes of b_i bits each, dv * b_i / 8 bytes;
+ *                          code j occupies bits [j b_i, (j + 1) b_i) of the
+ *                          row's little-endian bit string (bit p is bit p%8
+ *                          of byte p/8), as a b_i-bit two's complement value
+ *   padding up to a multiple of 128 bytes.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_NONFINITE 1
+#define ORC_BADARG 2
+
+static int q_of_bits(int b) { return (1 << (b - 1)) - 1; }
+
+static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8u; }
+
+static int bits_ok(int dk, int dv, const uint8_t *bits)
+{
+    for (int i = 0; i < dk; ++i) {
+        int b = bits[i];
+        if (b != 4 && b != 6 && b != 8) return 0;
+        if ((dv * b) % 8 != 0) return 0;
+    }
+    return 1;
+}
+
+size_t orc_page_bytes(int dk, int dv, const uint8_t *bits)
+{
+    size_t n = 4u * (size_t)dk;
+    for (int i = 0; i < dk; ++i) n += row_bytes(dv, bits[i]);
+    return (n + 127u) / 128u * 128u;
+}
+
+static size_t row_offset(int dk, int dv, const uint8_t *bits, int i)
+{
+    size_t n = 4u * (size_t)dk;
+    for (int t = 0; t < i; ++t) n += row_bytes(dv, bits[t]);
+    return n;
+}
+
+/* code j of a packed row, read one bit at a time, then sign-extended */
+static int32_t get_code(const uint8_t *row, int b, int j)
+{
+    uint32_t u = 0;
+    for (int t = 0; t < b; ++t) {
+        int p = j * b + t;
+        u |= (uint32_t)((row[p / 8] >> (p % 8)) & 1u) << t;
+    }
+    if (u & (1u << (b - 1))) return (int32_t)u - (int32_t)(1u << b);
+    return (int32_t)u;
+}
+
+static void put_code(uint8_t *row, int b, int j, int32_t z)
+{
+    uint32_t u = (uint32_t)z & ((1u << b) - 1u);
+    for (int t = 0; t < b; ++t) {
+        int p = j * b + t;
+        if ((u >> t) & 1u) row[p / 8] = (uint8_t)(row[p / 8] | (1u << (p % 8)));
+        else row[p / 8] = (uint8_t)(row[p / 8] & ~(1u << (p % 8)));
+    }
+}
+
+static float get_scale(const uint8_t *page, int i)
+{
+    float s;
+    memcpy(&s, page + 4 * (size_t)i, 4);
+    return s;
+}
+
+static void put_scale(uint8_t *page, int i, float s) { memcpy(page + 4 * (size_t)i, &s, 4); }
+
+/* exported for the pack/unpack pins */
+int32_t orc_get_code(const uint8_t *row, int b, int j) { return get_code(row, b, j); }
+void orc_put_code(uint8_t *row, int b, int j, int32_t z) { put_code(row, b, j, z); }
+
+/* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 */
+static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                        const uint8_t *page, double *S)
+{
+    for (int i = 0; i < dk; ++i) {
+        const uint8_t *row = page + row_offset(dk, dv, bits, i);
+        double s = (double)get_scale(page, i);
+        for (int j = 0; j < dv; ++j) {
+            int32_t z = get_code(row, bits[i], j);
+            S[(size_t)i * dv + j] = s * (double)r[i] * (double)c[j] * (double)z;
+        }
+    }
+}
+
+/*
+ * [bg-quant], [bg-smooth], [core], [steps] steps 4-6: quantise X row by row
+ * and write scales and codes into page.  quot (optional) receives the fp32
+ * quotient mu_ij / s_i that round() is applied to (for near-tie analysis).
+ * Returns ORC_NONFINITE if a row maximum is not finite.
+ */
+static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      const double *X, uint8_t *page, float *quot)
+{
+    int status = ORC_OK;
+    float *mu = (float *)malloc(sizeof(float) * (size_t)dv);
+    for (int i = 0; i < dk; ++i) {
+        int qb = q_of_bits(bits[i]);
+        float a = 0.0f;
+        for (int j = 0; j < dv; ++j) {
+            double rc = (double)r[i] * (double)c[j];
+            mu[j] = (float)(X[(size_t)i * dv + j] / rc);
+            float m = fabsf(mu[j]);
+            if (!(m <= a)) a = m; /* also propagates NaN */
+        }
+        if (!isfinite(a)) status = ORC_NONFINITE;
+        float s = a / (float)qb;
+        put_scale(page, i, s);
+        uint8_t *row = page + row_offset(dk, dv, bits, i);
+        for (int j = 0; j < dv; ++j) {
+            int32_t z = 0;
+            float x = 0.0f;
+            if (s > 0.0f && isfinite(s)) {
+                x = mu[j] / s;
+                float rz = rintf(x);
+                if (rz > (float)qb) rz = (float)qb;
+                if (rz < (float)-qb) rz = (float)-qb;
+                z = (int32_t)rz;
+            }
+            if (quot) quot[(size_t)i * dv + j] = x;
+            put_code(row, bits[i], j, z);
+        }
+    }
+    free(mu);
+    return status;
+}
+
+/* fp32 state -> packed page (the quantizer applied to a given state) */
+int orc_quantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      const float *S, uint8_t *page, float *quot)
+{
+    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
+    size_t nb = orc_page_bytes(dk, dv, bits);
+    memset(page, 0, nb);
+    double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    for (size_t e = 0; e < (size_t)dk * dv; ++e) X[e] = (double)S[e];
+    int st = requantize(dk, dv, bits, r, c, X, page, quot);
+    free(X);
+    return st;
+}
+
+/* packed page -> fp32 reconstruction fl32(s_i r_i c_j z_ij) */
+int orc_dequantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                        const uint8_t *page, float *S)
+{
+    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
+    double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    reconstruct(dk, dv, bits, r, c, page, X);
+    for (size_t e = 0; e < (size_t)dk * dv; ++e) S[e] = (float)X[e];
+    free(X);
+    return ORC_OK;
+}
+
+/*
+ * One quantized decode step of one unit ([steps] steps 1-6):
+ *   S^  = reconstruct(page_in)
+ *   P   = D S^,            D = diag(g)          ([bg-delta], [steps] step 2)
+ *   vo  = P^T k                                 (retrieval)
+ *   u   = beta (v - vo)
+ *   X   = P + k u^T                             (delta write)
+ *   y   = X^T q                                 ([steps] step 3, before requant)
+ *   page_out = requantize(X)
+ * y is returned in fp64; quot (optional, dk*dv floats) receives the fp32
+ * quotients the new codes were rounded from.
+ */
+int orc_step_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                  const uint8_t *page_in, uint8_t *page_out,
+                  const float *q, const float *k, const float *v, float beta, const float *g,
+                  double *y, float *quot)
+{
+    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
+    size_t nel = (size_t)dk * dv;
+    double *P = (double *)malloc(sizeof(double) * nel);
+    double *vo = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *u = (double *)malloc(sizeof(double) * (size_t)dv);
+    reconstruct(dk, dv, bits, r, c, page_in, P);
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) P[(size_t)i * dv + j] *= (double)g[i];
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += (double)k[i] * P[(size_t)i * dv + j];
+        vo[j] = acc;
+        u[j] = (double)beta * ((double)v[j] - acc);
+    }
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) P[(size_t)i * dv + j] += (double)k[i] * u[j]; /* P is now X */
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += (double)q[i] * P[(size_t)i * dv + j];
+        y[j] = acc;
+    }
+    memset(page_out, 0, orc_page_bytes(dk, dv, bits));
+    int st = requantize(dk, dv, bits, r, c, P, page_out, quot);
+    for (int j = 0; j < dv; ++j)
+        if (!isfinite(y[j])) st = ORC_NONFINITE;
+    free(P);
+    free(vo);
+    free(u);
+    return st;
+}
+
+/*
+ * The same recurrence with quantisation off, state kept in fp64 (in place):
+ *   X = D S + k (beta (v - (D S)^T k))^T,  y = X^T q,  S <- X.
+ */
+int orc_step_unit_f64(int dk, int dv, double *S, const float *q, const float *k,
+                      const float *v, float beta, const float *g, double *y)
+{
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] *= (double)g[i];
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += (double)k[i] * S[(size_t)i * dv + j];
+        double uj = (double)beta * ((double)v[j] - acc);
+        for (int i = 0; i < dk; ++i) S[(size_t)i * dv + j] += (double)k[i] * uj;
+    }
+    for (int j = 0; j < dv; ++j) {
+        double acc = 0.0;
+        for (int i = 0; i < dk; ++i) acc += (double)q[i] * S[(size_t)i * dv + j];
+        y[j] = acc;
+    }
+    return ORC_OK;
+}
+
+/*
+ * Many independent units at once (the CPU baseline): unit n uses head
+ * head[n] of the per-head tables bits [H][dk], r [H][dk], c [H][dv];
+ * its input page starts at pages_in + off_in[n], its output page at
+ * pages_out + off_out[n].  q, k, v, g: [n][128]; beta: [n]; y: [n][dv].
+ * Units are spread over nthreads OpenMP threads (<= 0: the runtime default).
+ * Returns the number of units that reported a non-finite value.
+ */
+int orc_step_many(int n, int dk, int dv, const int32_t *head, const uint8_t *bits,
+                  const float *r, const float *c, const uint8_t *pages_in, const int64_t *off_in,
+                  uint8_t *pages_out, const int64_t *off_out, const float *q, const float *k,
+                  const float *v, const float *beta, const float *g, double *y, int nthreads)
+{
+    int bad = 0;
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#else
+    nthreads = 1;
+#endif
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad) num_threads(nthreads)
+    for (int u = 0; u < n; ++u) {
+        int h = head[u];
+        int st = orc_step_unit(dk, dv, bits + (size_t)h * dk, r + (size_t)h * dk,
+                               c + (size_t)h * dv, pages_in + off_in[u], pages_out + off_out[u],
+                               q + (size_t)u * dk, k + (size_t)u * dk, v + (size_t)u * dv, beta[u],
+                               g + (size_t)u * dk, y + (size_t)u * dv, NULL);
+        if (st != ORC_OK) bad += 1;
+    }
+    return bad;
+}
+
+/* the number of OpenMP threads orc_step_many uses when nthreads <= 0 */
+int orc_default_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
