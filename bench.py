@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Benchmark: quantized gated delta-rule decode on B200.
+
+One step = one decode token over the whole batch of the workload (every
+(request, head) unit: unpack, dequantise, decay, retrieve, delta write,
+readout, requantise, repack), i.e. one launch of the fused decode kernel.
+
+Default workload: GDN with per-head 4/6/8-bit states averaging 6 bits,
+64 requests x 32 heads, d_k = d_v = 128, r, c ~ logU(0.25, 4), outlier
+initial state, inputs of a 256-token sequence (cycled when more steps are
+timed).  The L2 cache is flushed (a 384 MiB buffer is written) before every
+timed step, outside the timed interval, so each step reads its pages from
+HBM as it would in a 48-layer model.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank advances its own
+shard of requests (no data-path collective, weak scaling); the timed
+duration is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_linear_attention_decode_b200 import synth  # noqa: E402
+
+METRIC = "quantized-state decode head-steps/s and achieved HBM GB/s vs B200 peak"
+UNIT = "head-steps/s"
+L2_FLUSH_BYTES = 384 << 20
+DECODE_KERNEL = "decode_kernel"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+KERNEL_SRC = os.path.join(ROOT, "quantized_linear_attention_decode_b200", "csrc", "stq_kernels.cu")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--tokens", type=int, default=256, help="distinct input tokens (cycled)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the serving-pool sweep")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_sha() -> str:
+    return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(config: int):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    source is unchanged since it was taken; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    e = d.get(f"config{config}")
+    if not e or e.get("kernel_sha") != kernel_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def workload_info(wl):
+    rb = wl.row_bits().astype(np.int64)
+    per_head = [synth.algorithmic_bytes_per_head_step(wl.kind, int(rb[h].sum())) for h in range(wl.H)]
+    tables = wl.H * (2 * 128 * 4)  # r and c read once per head per launch
+    bytes_per_launch = wl.R * sum(per_head) + tables
+    return bytes_per_launch, float(rb.mean())
+
+
+# ---------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period: float = 0.01):
+        self.period = period
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                util = nv.nvmlDeviceGetUtilizationRates(self.h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        seen = 0
+        for s in busy:
+            seen |= s[1]
+        names = [n for n, bit in self.REASONS.items() if seen & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(busy)}
+
+
+# ---------------------------------------------------------------------- oracle (CPU baseline)
+
+
+class OracleRunner:
+    """The CPU oracle as it stands (OpenMP over units), set up on the first
+    `requests` requests of the workload (pages quantized by the oracle)."""
+
+    def __init__(self, config: int, seed: int, requests: int = 8):
+        import oracle as orc
+        self.orc = orc
+        wl = self.wl = synth.make_workload(config, seed=seed)
+        self.R = R = min(wl.R, requests)
+        self.rb = rb = wl.row_bits()
+        self.r, self.c = wl.row_factor.reshape(wl.H, 128), wl.col_factor.reshape(wl.H, 128)
+        S0 = wl.initial_state(np.arange(R))
+        sizes = [orc.page_bytes(rb[h]) for h in range(wl.H)]
+        head_off = np.concatenate([[0], np.cumsum(sizes)[:-1]])
+        slot = int(sum(sizes))
+        self.pages = np.zeros(R * slot, np.uint8)
+        for a in range(R):
+            for h in range(wl.H):
+                st = S0[a, h] if S0 is not None else np.zeros((128, 128), np.float32)
+                o = a * slot + head_off[h]
+                self.pages[o: o + sizes[h]] = orc.quantize_unit(rb[h], self.r[h], self.c[h], st)
+        self.head = np.tile(np.arange(wl.H, dtype=np.int32), R)
+        self.offs = (np.repeat(np.arange(R), wl.H) * slot + np.tile(head_off, R)).astype(np.int64)
+        self.threads = orc.default_threads()
+        self.inputs = {}
+
+    def _inp(self, t):
+        if t not in self.inputs:
+            wl, R = self.wl, self.R
+            inp = wl.step_inputs(t, np.arange(R))
+            g = inp["gate"]
+            g = np.repeat(g.reshape(R * wl.H, 1), 128, axis=1) if g.ndim == 2 else g.reshape(R * wl.H, 128)
+            self.inputs = {t: (inp["q"].reshape(-1, 128), inp["k"].reshape(-1, 128),
+                               inp["v"].reshape(-1, 128), inp["beta"].reshape(-1), np.ascontiguousarray(g))}
+        return self.inputs[t]
+
+    def step(self, t: int, units: int) -> float:
+        """Advances the first `units` units by token t; returns seconds."""
+        q, k, v, beta, g = self._inp(t)
+        u = min(units, len(self.head))
+        t0 = time.perf_counter()
+        out, _, _ = self.orc.step_many(self.head[:u], self.rb, self.r, self.c, self.pages,
+                                       self.offs[:u], self.offs[:u], len(self.pages), q[:u], k[:u],
+                                       v[:u], beta[:u], g[:u], self.threads)
+        dt = time.perf_counter() - t0
+        self.pages = out if u == len(self.head) else self._merge(out, u)
+        return dt
+
+    def _merge(self, out, u):
+        pages = self.pages.copy()
+        for n in range(u):
+            h = self.head[n]
+            o = self.offs[n]
+            nb = self.orc.page_bytes(self.rb[h])
+            pages[o: o + nb] = out[o: o + nb]
+        return pages
+
+
+def oracle_baseline(config: int, seed: int, seconds: float):
+    """Times the oracle on a bounded sample: consecutive tokens over all units
+    of its first requests until the time budget is spent."""
+    run = OracleRunner(config, seed)
+    units = len(run.head)
+    done, total, t = 0, 0.0, 0
+    while total < seconds:
+        total += run.step(t, units)
+        done += units
+        t += 1
+    sample = (f"{t} consecutive tokens x {run.R} requests x {run.wl.H} heads of {run.wl.name} "
+              f"({done} head-steps, {total:.1f} s of oracle time)")
+    return done / total, run.threads, sample
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return
+    run = OracleRunner(args.config, args.seed)
+    wl = run.wl
+    nsteps = args.warmup + args.steps
+    per_step_s = min(1.0, max(0.02, 150.0 / max(nsteps, 1)))
+    # size each step's sample of units to the per-step budget
+    dt = run.step(0, 8)
+    units = int(max(1, min(len(run.head), 8 * per_step_s / max(dt, 1e-6))))
+    done, total = 0, 0.0
+    for i in range(nsteps):
+        s = run.step(1 + i, units)
+        if i >= args.warmup:
+            total += s
+            done += units
+    value = done / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wl.R * wl.H / value, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64+f32", "data": "synthetic",
+        "config": {"workload": wl.name, "requests": wl.R, "heads": wl.H, "d_k": 128, "d_v": 128},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": run.threads, "kind": "oracle",
+                         "sample": f"{units} units of {wl.name} per step, {args.steps} timed steps "
+                                   f"({done} head-steps, {total:.1f} s)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- GPU arm
+
+
+def run_ours(args, rank: int, world: int):
+    import torch
+    from quantized_linear_attention_decode_b200 import stq
+
+    dev = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", dev))
+    wl = synth.make_workload(args.config, seed=args.seed + rank)
+    pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
+    req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
+    slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
+    S0 = wl.initial_state()
+    if S0 is not None:
+        stq.stq_quantize_state(pool, req, slot, torch.from_numpy(S0).cuda())
+        stq.stq_pool_check(pool)
+        del S0
+    ntok = max(1, args.tokens)
+    toks = []
+    for t in range(ntok):
+        inp = wl.step_inputs(t)
+        toks.append({k: torch.from_numpy(v).cuda() for k, v in inp.items()})
+    y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(t):
+        x = toks[t % ntok]
+        stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
+
+    for t in range(args.warmup):
+        flush.zero_()
+        step(t)
+    stq.stq_pool_check(pool, stream)
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    n0 = stq.stq_launch_count()
+    sampler = ClockSampler(dev)
+    with sampler:
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step(args.warmup + i)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    launches = stq.stq_launch_count() - n0
+    if dist:
+        dist.barrier()
+    stq.stq_pool_check(pool, stream)
+    times = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
+    total_ms = float(sum(times))
+    if dist:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    units = wl.R * wl.H
+    value = world * units * args.steps / (total_ms * 1e-3)
+    ms_per_step = total_ms / args.steps
+
+    bytes_per_launch, mean_bits = workload_info(wl)
+    kernel_s = statistics.mean(times) * 1e-3
+    peak, peak_kind = peaks()
+    achieved = bytes_per_launch / kernel_s / 1e9
+    traffic = recorded_traffic(args.config)
+
+    # ---- end to end through the public API: pinned host inputs in, y out
+    e2e = None
+    if args.e2e_steps > 0:
+        host = []
+        for t in range(min(ntok, 16)):
+            host.append({k: v.cpu().pin_memory() for k, v in toks[t].items()})
+        dev_in = {k: torch.empty_like(v) for k, v in toks[0].items()}
+        y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host[0].values())
+        d2h = y.numel() * y.element_size()
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.e2e_steps)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.e2e_steps)]
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.e2e_steps):
+            flush.zero_()
+            x = host[i % len(host)]
+            e_s[i].record(stream)
+            for k in dev_in:
+                dev_in[k].copy_(x[k], non_blocking=True)
+            stq.stq_decode_step(pool, req, slot, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["beta"],
+                                dev_in["gate"], y, stream)
+            y_host.copy_(y, non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
+        if dist:
+            tt = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e_ms = float(tt.item())
+        e2e = {"value": world * units * args.e2e_steps / (e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        stq.stq_pool_check(pool, stream)
+
+    sweep = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        sweep = pool_sweep(stq, flush, stream, peak)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, sample = oracle_baseline(args.config, args.seed, args.cpu_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample}
+
+    pool.close()
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "kind": "GDN" if wl.kind == synth.GDN else "KDA",
+                   "requests_per_gpu": wl.R, "heads": wl.H, "d_k": 128, "d_v": 128,
+                   "mean_bits": mean_bits, "slots": wl.S, "tokens_cycled": ntok,
+                   "l2": "flushed before every timed step (384 MiB write, outside the timed interval)",
+                   "parallelism": f"dp{world} (independent request shards)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": bytes_per_launch, "kernel": DECODE_KERNEL,
+                     "kernel_us": kernel_s * 1e6},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": sampler.summary(),
+        "pool_sweep": sweep,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def pool_sweep(stq, flush, stream, peak, reps: int = 20):
+    """Serving-pool sweep: R requests x 5 slots x 768 heads (48 layers x 16
+    heads), mixed 6-bit GDN, one token per launch over all heads; median
+    kernel time over `reps` launches with the L2 flushed before each."""
+    import torch
+    out = []
+    for R in (16, 32, 64, 128, 256):
+        wl = synth.make_workload(4, R=R)
+        pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
+        req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
+        slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
+        x = {k: torch.from_numpy(v).cuda() for k, v in wl.step_inputs(0).items()}
+        y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
+            e.record(stream)
+            if i >= 3:
+                ts.append((s, e))
+        torch.cuda.synchronize()
+        stq.stq_pool_check(pool, stream)
+        med = statistics.median(s.elapsed_time(e) for s, e in ts) * 1e-3
+        nbytes, _ = workload_info(wl)
+        packed, _ = stq.stq_pool_bytes(pool)
+        out.append({"requests": R, "heads": wl.H, "pool_gb": packed / 1e9, "touched_gb": nbytes / 1e9,
+                    "kernel_us": med * 1e6, "head_steps_per_s": wl.R * wl.H / med,
+                    "gbs": nbytes / med / 1e9, "frac": nbytes / med / 1e9 / peak})
+        pool.close()
+        del x, y
+        torch.cuda.empty_cache()
+    return out
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/*
+ * stq.h -- C ABI of the quantized gated delta-rule decode library (libstq.so).
+ *
+ * The library keeps the recurrent state of Gated DeltaNet (GDN) and Kimi
+ * Delta Attention (KDA) heads as bit-packed integer codes with per-row
+ * scales, and advances it one decode token at a time on an NVIDIA B200
+ * (sm_100a).  Method: "STEPQuant: When and Where Errors Matter in Delta-Rule
+ * Recurrent State Quantization" (paper.rainbus.top/paper/2609.38169);
+ * sections of that page are cited by name below.
+ *
+ * Conventions for every call:
+ *   - All entry points return an stq_status and never throw.  On a non-OK
+ *     return stq_last_error() gives a message (thread-local).
+ *   - Argument errors (null pointers, bad sizes, bad bit widths) are found
+ *     on the host, before anything is enqueued, and return STQ_ERR_ARG or
+ *     STQ_ERR_UNSUPPORTED; nothing is launched in that case.
+ *   - Work is asynchronous on the caller's CUDA stream, passed as a plain
+ *     pointer (a cudaStream_t / CUstream; NULL is the legacy default
+ *     stream).  Tensors named "device" must be device memory of the device
+ *     that was current when the pool was created, contiguous, row-major,
+ *     fp32 unless stated.  The caller owns every input and output buffer
+ *     and the stream; the pool owns its device memory and its copies of the
+ *     tables it was created from.
+ *   - Errors only the device can see (an out-of-range request or slot
+ *     index, a non-finite value) set a sticky error word in the pool; the
+ *     affected tile is skipped (index) or its content is unspecified
+ *     (non-finite).  stq_pool_check() reports and clears it.  No device
+ *     trap is ever raised.
+ *   - A call that names the same (request, slot) twice in its index lists
+ *     has undefined results (tiles are updated in place, one CTA each).
+ *   - Setting the environment variable STQ_FAULT=alloc makes
+ *     stq_pool_create fail with STQ_ERR_OOM, STQ_FAULT=launch makes every
+ *     launching call fail with STQ_ERR_CUDA, both before any CUDA call
+ *     (host-side fault injection for tests).
+ */
+#ifndef STQ_H
+#define STQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    STQ_OK = 0,
+    STQ_ERR_ARG = 1,         /* bad argument, found on the host */
+    STQ_ERR_OOM = 2,         /* device allocation failed */
+    STQ_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+    STQ_ERR_INDEX = 4,       /* device saw a request or slot index out of range */
+    STQ_ERR_NONFINITE = 5,   /* device saw a NaN or infinity */
+    STQ_ERR_UNSUPPORTED = 6, /* valid but not implemented (e.g. d_k != 128) */
+    STQ_ERR_TIMEOUT = 7      /* a bounded device-side wait gave up */
+} stq_status;
+
+typedef enum { STQ_GDN = 0, STQ_KDA = 1 } stq_kind;
+
+/* Opaque pool of packed states, owned by the library. */
+typedef struct stq_pool stq_pool;
+
+/*
+ * Pool description ("SGLang state pool" section: pool = concurrency x slots
+ * x per-request state).  A unit of precision ("core method" section: a whole
+ * head for GDN, one key row for KDA) carries a bit width b in {4, 6, 8}.
+ */
+typedef struct {
+    int32_t kind;         /* stq_kind */
+    int32_t num_requests; /* R >= 1 */
+    int32_t num_slots;    /* S >= 1 (five per request on the page's serving setup) */
+    int32_t num_heads;    /* H >= 1 */
+    int32_t d_k;          /* must be 128 ("linear attention and recurrent state": d_k = d_v = 128) */
+    int32_t d_v;          /* must be 128 */
+    const uint8_t *unit_bits;  /* host; GDN: [H] one width per head; KDA: [H * d_k] one per key row */
+    const float *row_factor;   /* host; [H * d_k] r_i, finite and > 0; NULL means all 1 */
+    const float *col_factor;   /* host; [H * d_v] c_j, finite and > 0; NULL means all 1 */
+} stq_pool_desc;
+
+/*
+ * Packed page of one (request, slot, head) state, in device memory:
+ *   bytes [0, 512)   128 fp32 scales s_i, one per key row
+ *   then rows i = 0..127 in order, row i holding 128 codes of b_i bits
+ *   (16 * b_i bytes); code j occupies bits [j b_i, (j+1) b_i) of the row's
+ *   little-endian bit string, as a b_i-bit two's complement integer in
+ *   [-q_b, q_b], q_b = 2^(b_i - 1) - 1
+ *   zero padding up to a multiple of 128 bytes.
+ * The pages of heads 0..H-1 follow each other inside a slot; slots are
+ * ordered [request][slot].  The state the page stands for is
+ *   S^_ij = s_i * r_i * c_j * z_ij          ("core method": X^ = r c z).
+ */
+
+/* Allocate a pool (device memory, all states zero) for the current device. */
+stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out);
+stq_status stq_pool_destroy(stq_pool *pool);
+
+/* Bytes of the whole packed pool and of one slot (all heads of one
+ * (request, slot)). */
+stq_status stq_pool_bytes(const stq_pool *pool, size_t *packed_bytes, size_t *per_slot_bytes);
+
+/* The same figures for a description, computed on the host without
+ * allocating anything (no device needed). */
+stq_status stq_desc_bytes(const stq_pool_desc *desc, size_t *packed_bytes, size_t *per_slot_bytes);
+
+/* Where head `head`'s page sits inside a slot, and its size in bytes. */
+stq_status stq_page_layout(const stq_pool *pool, int32_t head, size_t *offset_in_slot,
+                           size_t *page_bytes);
+
+/*
+ * Quantize fp32 states into the pool ("PTQ" section: Q(x) = s clip(round(x/s),
+ * -q_b, q_b), one absmax scale per key row of X / (r c)).
+ *   req_idx, slot_idx: device int32 [n]; entry e names the (request, slot)
+ *                      that state e is written to.
+ *   state:             device fp32 [n][H][128][128], S[i][j] with i the key row,
+ *                      16-byte aligned.
+ * n == 0 is a no-op.
+ */
+stq_status stq_quantize_state(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                              int32_t n, const float *state, void *stream);
+
+/* Reconstruct fp32 states fl32(s_i r_i c_j z_ij) from the pool into
+ * state_out (device fp32 [n][H][128][128], 16-byte aligned). */
+stq_status stq_dequantize_state(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, float *state_out, void *stream);
+
+/*
+ * One decode token for n (request, slot) entries and all H heads
+ * ("method steps", online decode, steps 1-7), updating the packed pages in
+ * place with no fp32 copy of the state kept anywhere:
+ *   S^  = reconstruct(page)                        step 1
+ *   X   = D S^ + beta k (v^T - k^T D S^)           step 2 ("gated delta rule")
+ *   y   = X^T q                                     step 3, before requantisation
+ *   page = pack(quantize_rows(X))                   steps 4-6
+ *   D = alpha I (GDN) or diag(d) (KDA).
+ *   q, k, v: device fp32 [n][H][128]; beta: device fp32 [n][H];
+ *   gate:    device fp32, GDN [n][H] (alpha), KDA [n][H][128] (d_i per key row);
+ *   y:       device fp32 [n][H][128], written.
+ * n == 0 is a no-op.
+ */
+stq_status stq_decode_step(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                           int32_t n, const float *q, const float *k, const float *v,
+                           const float *beta, const float *gate, float *y, void *stream);
+
+/* Copy one slot's raw pages (per_slot_bytes bytes) to / from host memory.
+ * Synchronous (device-wide ordering with the legacy default stream). */
+stq_status stq_export_slot(const stq_pool *pool, int32_t req, int32_t slot, void *host_dst,
+                           size_t bytes);
+stq_status stq_import_slot(stq_pool *pool, int32_t req, int32_t slot, const void *host_src,
+                           size_t bytes);
+
+/* Synchronize `stream`, then return and clear the pool's device error word
+ * (STQ_ERR_INDEX, STQ_ERR_NONFINITE or STQ_ERR_TIMEOUT; STQ_OK if clear). */
+stq_status stq_pool_check(stq_pool *pool, void *stream);
+
+/* Number of kernel launches this library has issued in this process. */
+uint64_t stq_launch_count(void);
+
+const char *stq_status_str(stq_status status);
+const char *stq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STQ_H */

@@ -1,0 +1,407 @@
+// stq_api.cu -- host side of the C ABI declared in include/stq.h:
+// pool allocation and tables, argument checking, status and error strings,
+// slot export/import, the device error word, host-side fault injection.
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "stq_internal.h"
+
+struct stq_pool {
+    int kind = 0, R = 0, S = 0, H = 0;
+    int device = 0;
+    size_t slot_bytes = 0, packed_bytes = 0;
+    uint8_t *d_pages = nullptr;
+    void *d_tables = nullptr;
+    uint32_t *d_err = nullptr;
+    stq::Tables t{};
+    std::vector<uint32_t> head_off, page_bytes;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+
+stq_status fail(stq_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+stq_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(e == cudaErrorMemoryAllocation ? STQ_ERR_OOM : STQ_ERR_CUDA, "%s: %s", what,
+                cudaGetErrorString(e));
+}
+
+bool fault(const char *which)
+{
+    const char *f = std::getenv("STQ_FAULT");
+    return f != nullptr && std::strcmp(f, which) == 0;
+}
+
+// Layout of one head's page from its row bit widths.
+struct HeadLayout {
+    uint32_t page_bytes;
+    uint16_t row_off[stq::kD];
+};
+
+HeadLayout head_layout(const uint8_t *row_bits)
+{
+    HeadLayout L{};
+    uint32_t off = stq::kScaleBytes;
+    for (int i = 0; i < stq::kD; ++i) {
+        L.row_off[i] = (uint16_t)off;
+        off += 16u * row_bits[i];
+    }
+    L.page_bytes = (off + stq::kPageAlign - 1) / stq::kPageAlign * stq::kPageAlign;
+    return L;
+}
+
+// Validates a description; fills the per-row bit table [H][128].
+stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
+{
+    if (d == nullptr) return fail(STQ_ERR_ARG, "desc is NULL");
+    if (d->kind != STQ_GDN && d->kind != STQ_KDA) return fail(STQ_ERR_ARG, "kind %d", d->kind);
+    if (d->num_requests < 1 || d->num_slots < 1 || d->num_heads < 1)
+        return fail(STQ_ERR_ARG, "sizes R=%d S=%d H=%d must be >= 1", d->num_requests,
+                    d->num_slots, d->num_heads);
+    if (d->d_k != stq::kD || d->d_v != stq::kD)
+        return fail(STQ_ERR_UNSUPPORTED, "d_k=%d d_v=%d: only 128 x 128 states", d->d_k, d->d_v);
+    if (d->unit_bits == nullptr) return fail(STQ_ERR_ARG, "unit_bits is NULL");
+    const int H = d->num_heads;
+    const size_t nunits = d->kind == STQ_GDN ? (size_t)H : (size_t)H * stq::kD;
+    for (size_t u = 0; u < nunits; ++u) {
+        int b = d->unit_bits[u];
+        if (b != 4 && b != 6 && b != 8)
+            return fail(STQ_ERR_ARG, "unit_bits[%zu] = %d (must be 4, 6 or 8)", u, b);
+    }
+    for (int which = 0; which < 2; ++which) {
+        const float *f = which ? d->col_factor : d->row_factor;
+        if (f == nullptr) continue;
+        for (size_t e = 0; e < (size_t)H * stq::kD; ++e)
+            if (!(std::isfinite(f[e]) && f[e] > 0.0f))
+                return fail(STQ_ERR_ARG, "%s_factor[%zu] = %g (must be finite and > 0)",
+                            which ? "col" : "row", e, (double)f[e]);
+    }
+    if (row_bits) {
+        row_bits->resize((size_t)H * stq::kD);
+        for (int h = 0; h < H; ++h)
+            for (int i = 0; i < stq::kD; ++i)
+                (*row_bits)[(size_t)h * stq::kD + i] =
+                    d->kind == STQ_GDN ? d->unit_bits[h] : d->unit_bits[(size_t)h * stq::kD + i];
+    }
+    return STQ_OK;
+}
+
+stq_status sizes_of(const stq_pool_desc *d, const std::vector<uint8_t> &row_bits,
+                    std::vector<uint32_t> *head_off, std::vector<uint32_t> *page_bytes,
+                    size_t *slot_bytes, size_t *packed)
+{
+    size_t off = 0;
+    for (int h = 0; h < d->num_heads; ++h) {
+        HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD]);
+        if (head_off) head_off->push_back((uint32_t)off);
+        if (page_bytes) page_bytes->push_back(L.page_bytes);
+        off += L.page_bytes;
+        if (off > 0xFFFFFFFFull) return fail(STQ_ERR_UNSUPPORTED, "slot larger than 4 GiB");
+    }
+    const double total = (double)off * d->num_requests * d->num_slots;
+    if (total > 9.0e18) return fail(STQ_ERR_ARG, "pool size overflows");
+    *slot_bytes = off;
+    *packed = off * (size_t)d->num_requests * (size_t)d->num_slots;
+    return STQ_OK;
+}
+
+stq::PoolView view(stq_pool *p)
+{
+    stq::PoolView v;
+    v.pages = p->d_pages;
+    v.slot_bytes = p->slot_bytes;
+    v.R = p->R;
+    v.S = p->S;
+    v.H = p->H;
+    v.kind = p->kind;
+    v.t = p->t;
+    v.err = p->d_err;
+    return v;
+}
+
+// Makes the pool's device current for the duration of a call.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev)
+    {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            ok = false;
+            return;
+        }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard()
+    {
+        int cur = -1;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+stq_status check_launch_args(const stq_pool *p, const int32_t *req, const int32_t *slot, int32_t n)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    if (n < 0) return fail(STQ_ERR_ARG, "n = %d", n);
+    if (n > 0 && (req == nullptr || slot == nullptr))
+        return fail(STQ_ERR_ARG, "req_idx / slot_idx is NULL");
+    if ((long long)n * p->H > 0x7FFFFFFFll) return fail(STQ_ERR_ARG, "n * H too large");
+    return STQ_OK;
+}
+
+}  // namespace
+
+namespace stq {
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace stq
+
+using stq::kD;
+
+extern "C" {
+
+const char *stq_status_str(stq_status s)
+{
+    switch (s) {
+    case STQ_OK: return "STQ_OK";
+    case STQ_ERR_ARG: return "STQ_ERR_ARG";
+    case STQ_ERR_OOM: return "STQ_ERR_OOM";
+    case STQ_ERR_CUDA: return "STQ_ERR_CUDA";
+    case STQ_ERR_INDEX: return "STQ_ERR_INDEX";
+    case STQ_ERR_NONFINITE: return "STQ_ERR_NONFINITE";
+    case STQ_ERR_UNSUPPORTED: return "STQ_ERR_UNSUPPORTED";
+    case STQ_ERR_TIMEOUT: return "STQ_ERR_TIMEOUT";
+    }
+    return "STQ_ERR_UNKNOWN";
+}
+
+const char *stq_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t stq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+stq_status stq_desc_bytes(const stq_pool_desc *desc, size_t *packed_bytes, size_t *per_slot_bytes)
+{
+    std::vector<uint8_t> rb;
+    stq_status st = check_desc(desc, &rb);
+    if (st != STQ_OK) return st;
+    size_t slot = 0, packed = 0;
+    st = sizes_of(desc, rb, nullptr, nullptr, &slot, &packed);
+    if (st != STQ_OK) return st;
+    if (packed_bytes) *packed_bytes = packed;
+    if (per_slot_bytes) *per_slot_bytes = slot;
+    return STQ_OK;
+}
+
+stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
+{
+    if (out == nullptr) return fail(STQ_ERR_ARG, "out is NULL");
+    *out = nullptr;
+    std::vector<uint8_t> rb;
+    stq_status st = check_desc(desc, &rb);
+    if (st != STQ_OK) return st;
+    if (fault("alloc")) return fail(STQ_ERR_OOM, "injected allocation failure (STQ_FAULT=alloc)");
+
+    stq_pool *p = new stq_pool();
+    p->kind = desc->kind;
+    p->R = desc->num_requests;
+    p->S = desc->num_slots;
+    p->H = desc->num_heads;
+    st = sizes_of(desc, rb, &p->head_off, &p->page_bytes, &p->slot_bytes, &p->packed_bytes);
+    if (st != STQ_OK) {
+        delete p;
+        return st;
+    }
+    const int H = p->H;
+    // host image of the tables
+    const size_t n_hoff = (size_t)H * 4, n_pb = (size_t)H * 4, n_ro = (size_t)H * kD * 2,
+                 n_rb = (size_t)H * kD, n_f = (size_t)H * kD * 4;
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t o_hoff = 0, o_pb = o_hoff + al(n_hoff), o_ro = o_pb + al(n_pb),
+                 o_rb = o_ro + al(n_ro), o_r = o_rb + al(n_rb), o_c = o_r + al(n_f),
+                 total = o_c + al(n_f);
+    std::vector<uint8_t> img(total, 0);
+    std::memcpy(&img[o_hoff], p->head_off.data(), n_hoff);
+    std::memcpy(&img[o_pb], p->page_bytes.data(), n_pb);
+    for (int h = 0; h < H; ++h) {
+        HeadLayout L = head_layout(&rb[(size_t)h * kD]);
+        std::memcpy(&img[o_ro + (size_t)h * kD * 2], L.row_off, kD * 2);
+    }
+    std::memcpy(&img[o_rb], rb.data(), n_rb);
+    float *fr = reinterpret_cast<float *>(&img[o_r]);
+    float *fc = reinterpret_cast<float *>(&img[o_c]);
+    for (size_t e = 0; e < (size_t)H * kD; ++e) {
+        fr[e] = desc->row_factor ? desc->row_factor[e] : 1.0f;
+        fc[e] = desc->col_factor ? desc->col_factor[e] : 1.0f;
+    }
+
+    cudaError_t e = cudaGetDevice(&p->device);
+    if (e != cudaSuccess) {
+        delete p;
+        return cuda_fail(e, "cudaGetDevice");
+    }
+    e = cudaMalloc(&p->d_pages, p->packed_bytes);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_tables, total);
+    if (e == cudaSuccess) e = cudaMalloc(&p->d_err, 256);
+    if (e == cudaSuccess) e = cudaMemset(p->d_pages, 0, p->packed_bytes);
+    if (e == cudaSuccess) e = cudaMemset(p->d_err, 0, 256);
+    if (e == cudaSuccess) e = cudaMemcpy(p->d_tables, img.data(), total, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+        stq_status r = cuda_fail(e, "pool allocation");
+        cudaFree(p->d_pages);
+        cudaFree(p->d_tables);
+        cudaFree(p->d_err);
+        cudaGetLastError();
+        delete p;
+        return r;
+    }
+    uint8_t *base = static_cast<uint8_t *>(p->d_tables);
+    p->t.head_off = reinterpret_cast<const uint32_t *>(base + o_hoff);
+    p->t.page_bytes = reinterpret_cast<const uint32_t *>(base + o_pb);
+    p->t.row_off = reinterpret_cast<const uint16_t *>(base + o_ro);
+    p->t.row_bits = base + o_rb;
+    p->t.r = reinterpret_cast<const float *>(base + o_r);
+    p->t.c = reinterpret_cast<const float *>(base + o_c);
+    *out = p;
+    return STQ_OK;
+}
+
+stq_status stq_pool_destroy(stq_pool *p)
+{
+    if (p == nullptr) return STQ_OK;
+    DeviceGuard g(p->device);
+    cudaFree(p->d_pages);
+    cudaFree(p->d_tables);
+    cudaFree(p->d_err);
+    delete p;
+    return STQ_OK;
+}
+
+stq_status stq_pool_bytes(const stq_pool *p, size_t *packed_bytes, size_t *per_slot_bytes)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    if (packed_bytes) *packed_bytes = p->packed_bytes;
+    if (per_slot_bytes) *per_slot_bytes = p->slot_bytes;
+    return STQ_OK;
+}
+
+stq_status stq_page_layout(const stq_pool *p, int32_t head, size_t *offset_in_slot,
+                           size_t *page_bytes)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    if (head < 0 || head >= p->H) return fail(STQ_ERR_ARG, "head %d out of [0, %d)", head, p->H);
+    if (offset_in_slot) *offset_in_slot = p->head_off[head];
+    if (page_bytes) *page_bytes = p->page_bytes[head];
+    return STQ_OK;
+}
+
+stq_status stq_quantize_state(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                              int32_t n, const float *state, void *stream)
+{
+    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && state == nullptr) return fail(STQ_ERR_ARG, "state is NULL");
+    if (reinterpret_cast<uintptr_t>(state) % 16 != 0) return fail(STQ_ERR_ARG, "state not 16-byte aligned");
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    cudaError_t e = stq::launch_quantize(view(p), req_idx, slot_idx, n, state, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "quantize launch");
+}
+
+stq_status stq_dequantize_state(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, float *state_out, void *stream)
+{
+    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && state_out == nullptr) return fail(STQ_ERR_ARG, "state_out is NULL");
+    if (reinterpret_cast<uintptr_t>(state_out) % 16 != 0)
+        return fail(STQ_ERR_ARG, "state_out not 16-byte aligned");
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    cudaError_t e =
+        stq::launch_dequantize(view(p), req_idx, slot_idx, n, state_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "dequantize launch");
+}
+
+stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                           int32_t n, const float *q, const float *k, const float *v,
+                           const float *beta, const float *gate, float *y, void *stream)
+{
+    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && (!q || !k || !v || !beta || !gate || !y))
+        return fail(STQ_ERR_ARG, "a q/k/v/beta/gate/y pointer is NULL");
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y};
+    cudaError_t e = stq::launch_decode(view(p), io, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "decode launch");
+}
+
+stq_status stq_export_slot(const stq_pool *p, int32_t req, int32_t slot, void *host_dst,
+                           size_t bytes)
+{
+    if (p == nullptr || host_dst == nullptr) return fail(STQ_ERR_ARG, "NULL argument");
+    if (req < 0 || req >= p->R || slot < 0 || slot >= p->S)
+        return fail(STQ_ERR_ARG, "(request %d, slot %d) out of range", req, slot);
+    if (bytes != p->slot_bytes)
+        return fail(STQ_ERR_ARG, "bytes = %zu, slot holds %zu", bytes, p->slot_bytes);
+    DeviceGuard g(p->device);
+    const uint8_t *src = p->d_pages + ((size_t)req * p->S + slot) * p->slot_bytes;
+    cudaError_t e = cudaMemcpy(host_dst, src, bytes, cudaMemcpyDeviceToHost);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "export");
+}
+
+stq_status stq_import_slot(stq_pool *p, int32_t req, int32_t slot, const void *host_src,
+                           size_t bytes)
+{
+    if (p == nullptr || host_src == nullptr) return fail(STQ_ERR_ARG, "NULL argument");
+    if (req < 0 || req >= p->R || slot < 0 || slot >= p->S)
+        return fail(STQ_ERR_ARG, "(request %d, slot %d) out of range", req, slot);
+    if (bytes != p->slot_bytes)
+        return fail(STQ_ERR_ARG, "bytes = %zu, slot holds %zu", bytes, p->slot_bytes);
+    DeviceGuard g(p->device);
+    uint8_t *dst = p->d_pages + ((size_t)req * p->S + slot) * p->slot_bytes;
+    cudaError_t e = cudaMemcpy(dst, host_src, bytes, cudaMemcpyHostToDevice);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "import");
+}
+
+stq_status stq_pool_check(stq_pool *p, void *stream)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    DeviceGuard g(p->device);
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    uint32_t word = 0;
+    e = cudaMemcpy(&word, p->d_err, 4, cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) e = cudaMemset(p->d_err, 0, 4);
+    if (e != cudaSuccess) return cuda_fail(e, "error word");
+    if (word & stq::kErrTimeout) return fail(STQ_ERR_TIMEOUT, "a device-side wait timed out");
+    if (word & stq::kErrIndex) return fail(STQ_ERR_INDEX, "request or slot index out of range");
+    if (word & stq::kErrNonFinite) return fail(STQ_ERR_NONFINITE, "non-finite value in the step");
+    return STQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// stq_internal.h -- shared between the host side (stq_api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "stq.h"
+
+namespace stq {
+
+constexpr int kD = 128;            // d_k = d_v
+constexpr int kScaleBytes = 4 * kD; // fp32 scales at the start of a page
+constexpr int kPageAlign = 128;    // pages are padded to this many bytes
+
+// device error word bits
+constexpr uint32_t kErrIndex = 1u;
+constexpr uint32_t kErrNonFinite = 2u;
+constexpr uint32_t kErrTimeout = 4u;
+
+// Per-head tables, one device allocation:
+//   head_off[H]    byte offset of the head's page inside a slot
+//   page_bytes[H]  size of the head's page
+//   row_off[H][128] byte offset of row i inside the page (scales come first)
+//   row_bits[H][128]
+//   r[H][128], c[H][128]
+struct Tables {
+    const uint32_t *head_off;
+    const uint32_t *page_bytes;
+    const uint16_t *row_off;
+    const uint8_t *row_bits;
+    const float *r;
+    const float *c;
+};
+
+struct PoolView {
+    uint8_t *pages;      // [R][S][slot_bytes]
+    size_t slot_bytes;
+    int R, S, H;
+    int kind;
+    Tables t;
+    uint32_t *err;
+};
+
+struct DecodeIO {
+    const int32_t *req_idx;
+    const int32_t *slot_idx;
+    int n;
+    const float *q, *k, *v, *beta, *gate;
+    float *y;
+};
+
+cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
+                            int n, const float *state, cudaStream_t stream);
+cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
+                              int n, float *state, cudaStream_t stream);
+
+void count_launch();
+
+}  // namespace stq

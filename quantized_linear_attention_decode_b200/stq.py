@@ -1,0 +1,241 @@
+"""Python binding of libstq.so (include/stq.h): argument marshalling only.
+
+Every function keeps the C name and forwards to the CUDA library; torch is
+used for device memory (``data_ptr()``) and streams (``cuda_stream``).  There
+is no fallback: if libstq.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libstq.so")
+
+STQ_GDN, STQ_KDA = 0, 1
+STATUS = {0: "STQ_OK", 1: "STQ_ERR_ARG", 2: "STQ_ERR_OOM", 3: "STQ_ERR_CUDA", 4: "STQ_ERR_INDEX",
+          5: "STQ_ERR_NONFINITE", 6: "STQ_ERR_UNSUPPORTED", 7: "STQ_ERR_TIMEOUT"}
+STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE, \
+    STQ_ERR_UNSUPPORTED, STQ_ERR_TIMEOUT = range(8)
+
+# every symbol include/stq.h declares
+EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
+           "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
+           "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
+           "stq_status_str", "stq_last_error")
+
+
+class StqError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class _Desc(C.Structure):
+    _fields_ = [("kind", C.c_int32), ("num_requests", C.c_int32), ("num_slots", C.c_int32),
+                ("num_heads", C.c_int32), ("d_k", C.c_int32), ("d_v", C.c_int32),
+                ("unit_bits", C.c_void_p), ("row_factor", C.c_void_p), ("col_factor", C.c_void_p)]
+
+
+_lib = None
+
+
+def load():
+    """Load libstq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m quantized_linear_attention_decode_b200.build`")
+    L = C.CDLL(LIB_PATH)
+    P, I32, SZ = C.c_void_p, C.c_int32, C.c_size_t
+    sig = {
+        "stq_pool_create": [P, P],
+        "stq_pool_destroy": [P],
+        "stq_pool_bytes": [P, P, P],
+        "stq_desc_bytes": [P, P, P],
+        "stq_page_layout": [P, I32, P, P],
+        "stq_quantize_state": [P, P, P, I32, P, P],
+        "stq_dequantize_state": [P, P, P, I32, P, P],
+        "stq_decode_step": [P, P, P, I32, P, P, P, P, P, P, P],
+        "stq_export_slot": [P, I32, I32, P, SZ],
+        "stq_import_slot": [P, I32, I32, P, SZ],
+        "stq_pool_check": [P, P],
+    }
+    for name, args in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = C.c_int
+    L.stq_launch_count.argtypes = []
+    L.stq_launch_count.restype = C.c_uint64
+    L.stq_status_str.argtypes = [C.c_int]
+    L.stq_status_str.restype = C.c_char_p
+    L.stq_last_error.argtypes = []
+    L.stq_last_error.restype = C.c_char_p
+    _lib = L
+    return L
+
+
+def _check(st: int) -> None:
+    if st != STQ_OK:
+        raise StqError(st, load().stq_last_error().decode())
+
+
+def _stream(stream) -> C.c_void_p:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return C.c_void_p(stream)
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype, shape=None, name="tensor"):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+def _desc(kind, R, S, H, unit_bits, row_factor, col_factor, keep):
+    ub = np.ascontiguousarray(unit_bits, np.uint8)
+    rf = None if row_factor is None else np.ascontiguousarray(row_factor, np.float32)
+    cf = None if col_factor is None else np.ascontiguousarray(col_factor, np.float32)
+    keep.extend([ub, rf, cf])
+    ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
+    return _Desc(int(kind), int(R), int(S), int(H), 128, 128, ptr(ub), ptr(rf), ptr(cf))
+
+
+class Pool:
+    """Owner of one stq_pool handle (destroyed with the object)."""
+
+    def __init__(self, handle, kind, R, S, H, unit_bits):
+        self.handle = handle
+        self.kind, self.R, self.S, self.H = kind, R, S, H
+        self.unit_bits = np.asarray(unit_bits, np.uint8).copy()
+
+    def __del__(self):
+        self.close()
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load().stq_pool_destroy(self.handle)
+            self.handle = None
+
+    @property
+    def row_bits(self) -> np.ndarray:
+        if self.kind == STQ_GDN:
+            return np.repeat(self.unit_bits.reshape(-1, 1), 128, axis=1)
+        return self.unit_bits.reshape(self.H, 128)
+
+    @property
+    def slot_bytes(self) -> int:
+        return stq_pool_bytes(self)[1]
+
+
+def stq_pool_create(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
+                    col_factor=None) -> Pool:
+    keep = []
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep)
+    h = C.c_void_p()
+    _check(load().stq_pool_create(C.byref(d), C.byref(h)))
+    return Pool(h, kind, num_requests, num_slots, num_heads, unit_bits)
+
+
+def stq_pool_destroy(pool: Pool) -> None:
+    pool.close()
+
+
+def stq_pool_bytes(pool: Pool):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(load().stq_pool_bytes(pool.handle, C.byref(a), C.byref(b)))
+    return a.value, b.value
+
+
+def stq_desc_bytes(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
+                   col_factor=None):
+    keep = []
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep)
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(load().stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)))
+    return a.value, b.value
+
+
+def stq_page_layout(pool: Pool, head: int):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(load().stq_page_layout(pool.handle, int(head), C.byref(a), C.byref(b)))
+    return a.value, b.value
+
+
+def _idx(pool, req_idx, slot_idx):
+    import torch
+    n = int(req_idx.numel())
+    return (n, _dev(req_idx, torch.int32, (n,), "req_idx"), _dev(slot_idx, torch.int32, (n,), "slot_idx"))
+
+
+def stq_quantize_state(pool: Pool, req_idx, slot_idx, state, stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    st = _dev(state, torch.float32, (n, pool.H, 128, 128), "state")
+    _check(load().stq_quantize_state(pool.handle, r, s, n, st, _stream(stream)))
+
+
+def stq_dequantize_state(pool: Pool, req_idx, slot_idx, state_out, stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    st = _dev(state_out, torch.float32, (n, pool.H, 128, 128), "state_out")
+    _check(load().stq_dequantize_state(pool.handle, r, s, n, st, _stream(stream)))
+
+
+def stq_decode_step(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    f = torch.float32
+    vec = (n, pool.H, 128)
+    gshape = (n, pool.H) if pool.kind == STQ_GDN else vec
+    _check(load().stq_decode_step(
+        pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
+        _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
+        _stream(stream)))
+
+
+def stq_export_slot(pool: Pool, req: int, slot: int) -> np.ndarray:
+    nb = pool.slot_bytes
+    out = np.empty(nb, np.uint8)
+    _check(load().stq_export_slot(pool.handle, int(req), int(slot), out.ctypes.data, nb))
+    return out
+
+
+def stq_import_slot(pool: Pool, req: int, slot: int, data) -> None:
+    data = np.ascontiguousarray(data, np.uint8)
+    _check(load().stq_import_slot(pool.handle, int(req), int(slot), data.ctypes.data, data.nbytes))
+
+
+def stq_pool_check(pool: Pool, stream=None, raise_on_error: bool = True) -> int:
+    st = load().stq_pool_check(pool.handle, _stream(stream))
+    if raise_on_error:
+        _check(st)
+    return st
+
+
+def stq_launch_count() -> int:
+    return int(load().stq_launch_count())
+
+
+def stq_status_str(status: int) -> str:
+    return load().stq_status_str(int(status)).decode()
+
+
+def stq_last_error() -> str:
+    return load().stq_last_error().decode()

@@ -1,0 +1,119 @@
+"""Host-side checks of libstq.so that need no GPU: it loads, exports every
+symbol include/stq.h declares, validates arguments, reproduces the pool
+accounting, and injects faults on the host."""
+import ctypes as C
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as orc
+from pages import decode_page, page_bytes, row_offsets
+from quantized_linear_attention_decode_b200 import stq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "stq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(stq_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = stq.load()
+    names = _declared()
+    assert "stq_decode_step" in names and len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(stq.EXPORTS)
+
+
+def test_status_strings():
+    for code, name in stq.STATUS.items():
+        assert stq.stq_status_str(code) == name
+
+
+def test_desc_bytes_reproduces_pool_formula():
+    """pool = requests x slots x per-slot state ("SGLang state pool"); a
+    page is 512 B of fp32 scales + 16 b bytes per row, padded to 128 B."""
+    rng = np.random.default_rng(0)
+    bits = rng.choice(np.array([4, 6, 8], np.uint8), 48)
+    packed, slot = stq.stq_desc_bytes(stq.STQ_GDN, 7, 5, 48, bits)
+    assert slot == sum(512 + 2048 * int(b) for b in bits)
+    assert packed == 7 * 5 * slot
+    kbits = rng.choice(np.array([4, 6, 8], np.uint8), 3 * 128)
+    packed, slot = stq.stq_desc_bytes(stq.STQ_KDA, 2, 1, 3, kbits)
+    assert slot == sum(page_bytes(kbits[h * 128:(h + 1) * 128]) for h in range(3))
+    # the page's serving setting: batch 512, 5 slots, 2304 GDN heads of 128 x 128
+    packed, _ = stq.stq_desc_bytes(stq.STQ_GDN, 512, 5, 2304, np.full(2304, 6, np.uint8))
+    fp32 = 512 * 5 * 2304 * 128 * 128 * 4
+    assert fp32 == 360 * 2 ** 30
+    bits_per_value = packed * 8 / (512 * 5 * 2304 * 128 * 128)
+    assert bits_per_value == 6.25  # 6-bit codes + one fp32 scale per 128 values
+    assert abs(fp32 / packed - 32 / 6.25) < 1e-12
+
+
+@pytest.mark.parametrize("bad", [
+    dict(unit_bits=np.array([6, 5], np.uint8)),
+    dict(kind=3),
+    dict(R=0),
+    dict(row_factor=np.array([1.0] * 255 + [0.0], np.float32)),
+    dict(col_factor=np.array([1.0] * 255 + [np.nan], np.float32)),
+])
+def test_desc_validation(bad):
+    args = dict(kind=stq.STQ_GDN, R=1, S=1, H=2, unit_bits=np.array([6, 8], np.uint8),
+                row_factor=None, col_factor=None)
+    args.update(bad)
+    with pytest.raises(stq.StqError) as e:
+        stq.stq_desc_bytes(args["kind"], args["R"], args["S"], args["H"], args["unit_bits"],
+                           args["row_factor"], args["col_factor"])
+    assert e.value.status == stq.STQ_ERR_ARG
+
+
+def test_unsupported_head_dim():
+    L = stq.load()
+    ub = np.array([6], np.uint8)
+    d = stq._Desc(0, 1, 1, 1, 64, 64, ub.ctypes.data, None, None)
+    a, b = C.c_size_t(), C.c_size_t()
+    assert L.stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)) == stq.STQ_ERR_UNSUPPORTED
+
+
+def test_null_arguments_rejected_before_any_cuda_call():
+    L = stq.load()
+    assert L.stq_pool_create(None, None) == stq.STQ_ERR_ARG
+    assert L.stq_decode_step(None, None, None, 0, None, None, None, None, None, None, None) == stq.STQ_ERR_ARG
+    assert L.stq_pool_check(None, None) == stq.STQ_ERR_ARG
+    assert L.stq_export_slot(None, 0, 0, None, 0) == stq.STQ_ERR_ARG
+
+
+def test_fault_injection_alloc(monkeypatch):
+    monkeypatch.setenv("STQ_FAULT", "alloc")
+    with pytest.raises(stq.StqError) as e:
+        stq.stq_pool_create(stq.STQ_GDN, 1, 1, 1, np.array([8], np.uint8))
+    assert e.value.status == stq.STQ_ERR_OOM
+    assert "injected" in stq.stq_last_error()
+
+
+def test_page_reader_agrees_with_oracle_packer():
+    """The tests' vectorised page reader and the oracle's bit-by-bit packer
+    read the same bytes the same way."""
+    rng = np.random.default_rng(9)
+    bits = rng.choice(np.array([4, 6, 8], np.uint8), 128)
+    page = np.zeros(page_bytes(bits), np.uint8)
+    assert len(page) == orc.page_bytes(bits)
+    np.testing.assert_array_equal(row_offsets(bits), orc.row_offsets(bits))
+    want = np.zeros((128, 128), np.int32)
+    offs = row_offsets(bits)
+    for i, b in enumerate(bits):
+        q = (1 << (int(b) - 1)) - 1
+        want[i] = rng.integers(-q, q + 1, 128)
+        row = np.zeros(16 * int(b), np.uint8)
+        for j in range(128):
+            orc.put_code(row, int(b), j, int(want[i, j]))
+        page[offs[i]: offs[i] + len(row)] = row
+    page[:512] = np.arange(128, dtype=np.float32).view(np.uint8)
+    s, z = decode_page(page, bits)
+    np.testing.assert_array_equal(z, want)
+    np.testing.assert_array_equal(s, np.arange(128, dtype=np.float32))
