@@ -92,6 +92,29 @@ def workload_info(wl):
     return bytes_per_launch, float(rb.mean())
 
 
+# ---------------------------------------------------------------------- ranks
+
+
+def rank_world(args):
+    """(rank, world size) from the torchrun environment; 1 process otherwise."""
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+
+
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank advances its own shard of requests, drawn from its own seed."""
+    return base_seed + 1000003 * rank
+
+
+def max_over_ranks(x: float, dist=None, device: str = "cpu") -> float:
+    """The slowest rank's value (every rank calls this once per quantity)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------- clocks
 
 
@@ -276,7 +299,7 @@ def run_ours(args, rank: int, world: int):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", dev))
-    wl = synth.make_workload(args.config, seed=args.seed + rank)
+    wl = synth.make_workload(args.config, seed=shard_seed(args.seed, rank))
     pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
     req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
     slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
@@ -322,11 +345,7 @@ def run_ours(args, rank: int, world: int):
         dist.barrier()
     stq.stq_pool_check(pool, stream)
     times = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
-    total_ms = float(sum(times))
-    if dist:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(float(sum(times)), dist, "cuda")
     units = wl.R * wl.H
     value = world * units * args.steps / (total_ms * 1e-3)
     ms_per_step = total_ms / args.steps
@@ -363,11 +382,7 @@ def run_ours(args, rank: int, world: int):
             y_host.copy_(y, non_blocking=True)
             e_e[i].record(stream)
         torch.cuda.synchronize()
-        e_ms = float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)))
-        if dist:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
+        e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))), dist, "cuda")
         e2e = {"value": world * units * args.e2e_steps / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         stq.stq_pool_check(pool, stream)
@@ -447,8 +462,7 @@ def pool_sweep(stq, flush, stream, peak, reps: int = 20):
 
 def main():
     args = parse()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", str(args.gpus if args.gpus == 1 else 1)))
+    rank, world = rank_world(args)
     if args.impl == "reference":
         run_reference(args, rank, world)
     else:
