@@ -131,8 +131,9 @@ stq_status stq_dequantize_state(stq_pool *pool, const int32_t *req_idx, const in
  *   y   = X^T q                                     step 3, before requantisation
  *   page = pack(quantize_rows(X))                   steps 4-6
  *   D = alpha I (GDN) or diag(d) (KDA).
- *   q, k, v: device fp32 [n][H][128]; beta: device fp32 [n][H];
- *   gate:    device fp32, GDN [n][H] (alpha), KDA [n][H][128] (d_i per key row);
+ *   q, k, v: device fp32 [n][H][128], 16-byte aligned; beta: device fp32 [n][H];
+ *   gate:    device fp32, GDN [n][H] (alpha), KDA [n][H][128] (d_i per key row,
+ *            16-byte aligned);
  *   y:       device fp32 [n][H][128], written.
  * n == 0 is a no-op.
  */

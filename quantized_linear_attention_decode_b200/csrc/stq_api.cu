@@ -233,9 +233,10 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     const size_t n_hoff = (size_t)H * 4, n_pb = (size_t)H * 4, n_ro = (size_t)H * kD * 2,
                  n_rb = (size_t)H * kD, n_f = (size_t)H * kD * 4;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t n_blk = (size_t)H * stq::kHeadBlock;
     const size_t o_hoff = 0, o_pb = o_hoff + al(n_hoff), o_ro = o_pb + al(n_pb),
                  o_rb = o_ro + al(n_ro), o_r = o_rb + al(n_rb), o_c = o_r + al(n_f),
-                 total = o_c + al(n_f);
+                 o_blk = o_c + al(n_f), total = o_blk + al(n_blk);
     std::vector<uint8_t> img(total, 0);
     std::memcpy(&img[o_hoff], p->head_off.data(), n_hoff);
     std::memcpy(&img[o_pb], p->page_bytes.data(), n_pb);
@@ -249,6 +250,13 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     for (size_t e = 0; e < (size_t)H * kD; ++e) {
         fr[e] = desc->row_factor ? desc->row_factor[e] : 1.0f;
         fc[e] = desc->col_factor ? desc->col_factor[e] : 1.0f;
+    }
+    for (int h = 0; h < H; ++h) {
+        uint8_t *blk = &img[o_blk + (size_t)h * stq::kHeadBlock];
+        std::memcpy(blk, fr + (size_t)h * kD, kD * 4);
+        std::memcpy(blk + 512, fc + (size_t)h * kD, kD * 4);
+        std::memcpy(blk + 1024, &img[o_ro + (size_t)h * kD * 2], kD * 2);
+        std::memcpy(blk + 1280, &rb[(size_t)h * kD], kD);
     }
 
     cudaError_t e = cudaGetDevice(&p->device);
@@ -278,6 +286,7 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->t.row_bits = base + o_rb;
     p->t.r = reinterpret_cast<const float *>(base + o_r);
     p->t.c = reinterpret_cast<const float *>(base + o_c);
+    p->t.block = base + o_blk;
     *out = p;
     return STQ_OK;
 }
@@ -351,6 +360,12 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
     if (st != STQ_OK) return st;
     if (n > 0 && (!q || !k || !v || !beta || !gate || !y))
         return fail(STQ_ERR_ARG, "a q/k/v/beta/gate/y pointer is NULL");
+    {
+        const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                              reinterpret_cast<uintptr_t>(v) |
+                              (p != nullptr && p->kind == STQ_KDA ? reinterpret_cast<uintptr_t>(gate) : 0);
+        if (mis % 16 != 0) return fail(STQ_ERR_ARG, "q, k, v (and the KDA gate) must be 16-byte aligned");
+    }
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
