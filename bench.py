@@ -41,7 +41,7 @@ UNIT = "head-steps/s"
 L2_FLUSH_BYTES = 384 << 20
 DECODE_KERNEL = "decode_kernel"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
-KERNEL_SRC = os.path.join(ROOT, "quantized_linear_attention_decode_b200", "csrc", "stq_kernels.cu")
+KERNEL_SRC = os.path.join(ROOT, "quantized_linear_attention_decode_b200", "csrc", "stq_decode.cu")
 
 
 def parse():

@@ -129,9 +129,13 @@ class Pool:
         self.close()
 
     def close(self):
-        if getattr(self, "handle", None):
-            load().stq_pool_destroy(self.handle)
-            self.handle = None
+        h = getattr(self, "handle", None)
+        self.handle = None
+        if h and _lib is not None:
+            try:
+                _lib.stq_pool_destroy(h)
+            except Exception:  # noqa: BLE001  (interpreter shutdown)
+                pass
 
     @property
     def row_bits(self) -> np.ndarray:
