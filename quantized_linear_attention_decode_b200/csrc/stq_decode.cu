@@ -66,7 +66,8 @@ struct __align__(16) RowCoef {
 struct __align__(128) Smem {
     Stage st[kStages];
     RowCoef rc[2];
-    float red[2048];   // column partial sums [8 warps][v, y][128]
+    float red[2048];   // column partial sums [8 warps][v, y][128]; then row-max partials
+    float rowinv[kD];  // per-row quantisation multiplier (pass 2)
     float ut[kD];      // u_j / c_j
     uint8_t *stage_page[kStages];
     uint32_t stage_valid[kStages];
@@ -218,21 +219,42 @@ __device__ __forceinline__ float rcp_approx(float x)
 
 __device__ __forceinline__ float f_of(uint32_t u) { return __uint_as_float(u); }
 
+// (a & m) ^ c | (c & ~m) in one LOP3: keep a's bits under mask m, flip those
+// set in c, and take c's bits elsewhere.
+template <uint32_t M, uint32_t C>
+__device__ __forceinline__ uint32_t masked_field(uint32_t a)
+{
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "n"(M), "n"(C));
+    return d;
+}
+
 // ---------------------------------------------------------------- codecs
 //
 // unpack: the 8 codes of columns [8 cg, 8 cg + 8) of one packed row (in
 // shared memory) as float pairs (first pass).  The b-bit two's complement code z becomes
-// the offset code u = z + 2^(b-1) (one XOR per word), u is placed in the
-// mantissa of 2^23 (exact: 2^23 + u) and 2^23 + 2^(b-1) is subtracted
-// (exact).
+// the offset code u = z + 2^(b-1) by flipping its top bit, u is placed in the
+// mantissa of a power of two 2^E whose last mantissa bit weighs 1 (exact: 2^E + u)
+// and 2^E + 2^(b-1) is subtracted (exact).  For 4 and 6 bits one LOP3 per code
+// masks the field where it lies in the word, flips its top bit and sets the
+// exponent: a field at bit offset f takes E = 23 - f, so no shifts are needed
+// for fields that end below bit 23.
 //
-// Requantised codes come back as the bit patterns of fl(w inv + kMagicOut):
-// 2^23 + u for 4 and 6 bits, 1.5 * 2^23 + z for 8 bits (packed by Chunk<B>).
+// store: the inverse, straight to the page in global memory, for requantised
+// codes given as the bit patterns of fl(w inv + kMagicOut): 2^23 + u for 4
+// and 6 bits, 1.5 * 2^23 + z for 8 bits.
 
 template <int B> struct Codec;
 
 template <> struct Codec<8> {
     static constexpr float kMagicOut = 12582912.0f;  // 1.5 * 2^23: low byte = z (two's complement)
+    __device__ __forceinline__ static void store(uint8_t *rowg, int cg, const uint32_t b[8])
+    {
+        uint2 w;
+        w.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+        w.y = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+        *reinterpret_cast<uint2 *>(rowg + cg * 8) = w;
+    }
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
         const uint2 w = *reinterpret_cast<const uint2 *>(rowp + cg * 8);
@@ -247,23 +269,47 @@ template <> struct Codec<8> {
 
 template <> struct Codec<4> {
     static constexpr float kMagicOut = 8388616.0f;  // 2^23 + 8: mantissa = u = z + 8 in [1, 15]
+    __device__ __forceinline__ static void store(uint8_t *rowg, int cg, const uint32_t b[8])
+    {
+        // b[t] = 0x4B000000 + u_t: sum_t b[t] 16^t = sum_t u_t 16^t + 0xFB000000 (mod 2^32)
+        uint32_t acc = b[0];
+#pragma unroll
+        for (int t = 1; t < 8; ++t) acc += b[t] << (4 * t);
+        *reinterpret_cast<uint32_t *>(rowg + cg * 4) = (acc - 0xFB000000u) ^ 0x88888888u;
+    }
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
-        const uint32_t x = *reinterpret_cast<const uint32_t *>(rowp + cg * 4) ^ 0x88888888u;
-        const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
-        const float2 off = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
-        z[0] = fadd2(make_float2(f_of(__byte_perm(lo, 0x4B000000u, 0x7650)), f_of(__byte_perm(hi, 0x4B000000u, 0x7650))), off);
-        z[1] = fadd2(make_float2(f_of(__byte_perm(lo, 0x4B000000u, 0x7651)), f_of(__byte_perm(hi, 0x4B000000u, 0x7651))), off);
-        z[2] = fadd2(make_float2(f_of(__byte_perm(lo, 0x4B000000u, 0x7652)), f_of(__byte_perm(hi, 0x4B000000u, 0x7652))), off);
-        z[3] = fadd2(make_float2(f_of(__byte_perm(lo, 0x4B000000u, 0x7653)), f_of(__byte_perm(hi, 0x4B000000u, 0x7653))), off);
+        // code t at bits [4t, 4t + 4); codes 5..7 are shifted down to offsets 0, 4, 8
+        const uint32_t x = *reinterpret_cast<const uint32_t *>(rowp + cg * 4);
+        const uint32_t t = x >> 20;
+        const uint32_t c0 = masked_field<0xFu, 0x4B000008u>(x);       // 2^23 + u
+        const uint32_t c1 = masked_field<0xF0u, 0x49000080u>(x);      // 2^19 + u
+        const uint32_t c2 = masked_field<0xF00u, 0x47000800u>(x);     // 2^15 + u
+        const uint32_t c3 = masked_field<0xF000u, 0x45008000u>(x);    // 2^11 + u
+        const uint32_t c4 = masked_field<0xF0000u, 0x43080000u>(x);   // 2^7 + u
+        const uint32_t c5 = masked_field<0xFu, 0x4B000008u>(t);
+        const uint32_t c6 = masked_field<0xF0u, 0x49000080u>(t);
+        const uint32_t c7 = masked_field<0xF00u, 0x47000800u>(t);
+        z[0] = fadd2(make_float2(f_of(c0), f_of(c1)), make_float2(-8388616.0f, -524296.0f));
+        z[1] = fadd2(make_float2(f_of(c2), f_of(c3)), make_float2(-32776.0f, -2056.0f));
+        z[2] = fadd2(make_float2(f_of(c4), f_of(c5)), make_float2(-136.0f, -8388616.0f));
+        z[3] = fadd2(make_float2(f_of(c6), f_of(c7)), make_float2(-524296.0f, -32776.0f));
     }
 };
 
 template <> struct Codec<6> {
     static constexpr float kMagicOut = 8388640.0f;  // 2^23 + 32: mantissa = u = z + 32 in [1, 63]
-    __device__ __forceinline__ static uint32_t field(uint32_t a)
+    __device__ __forceinline__ static void store(uint8_t *rowg, int cg, const uint32_t b[8])
     {
-        return ((a ^ 0x20u) & 0x3Fu) | 0x4B000000u;
+        // b[t] = 0x4B000000 + u_t; the 0x4B000000 parts cancel or shift out except a constant
+        uint32_t lo = b[0] + (b[1] << 6) + (b[2] << 12) + (b[3] << 18) + (b[4] << 24) + (b[5] << 30);
+        lo = (lo - 0x0B000000u) ^ 0x20820820u;
+        const uint32_t hi = ((b[5] >> 2) + (b[6] << 4) + (b[7] << 10)) ^ 0x8208u;
+        // 6 bytes at 6 cg: a 4-byte and a 2-byte store, both aligned
+        const uint32_t odd = cg & 1;
+        uint8_t *p = rowg + cg * 6;
+        *reinterpret_cast<uint32_t *>(p + 2 * odd) = odd ? (lo >> 16) | (hi << 16) : lo;
+        *reinterpret_cast<uint16_t *>(p + 4 * (1 - odd)) = static_cast<uint16_t>(odd ? lo : hi);
     }
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
@@ -274,11 +320,20 @@ template <> struct Codec<6> {
         const uint32_t w1 = *reinterpret_cast<const uint32_t *>(rowp + base + 4);
         const uint32_t lo = __funnelshift_r(w0, w1, sh);
         const uint32_t hi = w1 >> sh;
-        const float2 off = make_float2(-8388640.0f, -8388640.0f);  // -(2^23 + 32)
-        z[0] = fadd2(make_float2(f_of(field(lo)), f_of(field(lo >> 6))), off);
-        z[1] = fadd2(make_float2(f_of(field(lo >> 12)), f_of(field(lo >> 18))), off);
-        z[2] = fadd2(make_float2(f_of(field(lo >> 24)), f_of(field(__funnelshift_r(lo, hi, 30)))), off);
-        z[3] = fadd2(make_float2(f_of(field(hi >> 4)), f_of(field(hi >> 10))), off);
+        const uint32_t x = lo >> 18;                     // codes 3, 4 at offsets 0, 6
+        const uint32_t y = __funnelshift_r(lo, hi, 30);  // codes 5, 6, 7 at offsets 0, 6, 12
+        const uint32_t c0 = masked_field<0x3Fu, 0x4B000020u>(lo);     // 2^23 + u
+        const uint32_t c1 = masked_field<0xFC0u, 0x48000800u>(lo);    // 2^17 + u
+        const uint32_t c2 = masked_field<0x3F000u, 0x45020000u>(lo);  // 2^11 + u
+        const uint32_t c3 = masked_field<0x3Fu, 0x4B000020u>(x);
+        const uint32_t c4 = masked_field<0xFC0u, 0x48000800u>(x);
+        const uint32_t c5 = masked_field<0x3Fu, 0x4B000020u>(y);
+        const uint32_t c6 = masked_field<0xFC0u, 0x48000800u>(y);
+        const uint32_t c7 = masked_field<0x3F000u, 0x45020000u>(y);
+        z[0] = fadd2(make_float2(f_of(c0), f_of(c1)), make_float2(-8388640.0f, -131104.0f));
+        z[1] = fadd2(make_float2(f_of(c2), f_of(c3)), make_float2(-2080.0f, -8388640.0f));
+        z[2] = fadd2(make_float2(f_of(c4), f_of(c5)), make_float2(-131104.0f, -8388640.0f));
+        z[3] = fadd2(make_float2(f_of(c6), f_of(c7)), make_float2(-131104.0f, -2080.0f));
     }
 };
 
@@ -289,122 +344,31 @@ __device__ __forceinline__ void unpack_any(int b, const uint8_t *rowp, int cg, f
     else Codec<4>::unpack(rowp, cg, z);
 }
 
+__device__ __forceinline__ void store_any(int b, uint8_t *rowg, int cg, const uint32_t bits[8])
+{
+    if (b == 8) Codec<8>::store(rowg, cg, bits);
+    else if (b == 6) Codec<6>::store(rowg, cg, bits);
+    else Codec<4>::store(rowg, cg, bits);
+}
+
 __device__ __forceinline__ float magic_out(int b)
 {
     return b == 8 ? Codec<8>::kMagicOut : (b == 6 ? Codec<6>::kMagicOut : Codec<4>::kMagicOut);
 }
 
 
-// ---------------------------------------------------------------- 32-code chunks
-//
-// The second pass gives each row to a quad of lanes: lane q of the quad owns
-// columns [32 q, 32 q + 32), i.e. the chunk of 4 b bytes at row offset 4 b q.
-
-template <int B> struct Chunk;
-
-template <> struct Chunk<8> {
-    __device__ __forceinline__ static void unpack(const uint8_t *rowp, int q, float2 z[16])
-    {
-        const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 32 * q);
-        const uint4 b = *reinterpret_cast<const uint4 *>(rowp + 32 * q + 16);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-        const float2 off = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const uint32_t x = w[k] ^ 0x80808080u;
-            z[2 * k] = fadd2(make_float2(f_of(__byte_perm(x, 0x4B000000u, 0x7650)), f_of(__byte_perm(x, 0x4B000000u, 0x7651))), off);
-            z[2 * k + 1] = fadd2(make_float2(f_of(__byte_perm(x, 0x4B000000u, 0x7652)), f_of(__byte_perm(x, 0x4B000000u, 0x7653))), off);
-        }
-    }
-    __device__ __forceinline__ static void store(uint8_t *rowg, int q, const uint32_t b[32])
-    {
-        uint32_t w[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-            w[k] = __byte_perm(__byte_perm(b[4 * k], b[4 * k + 1], 0x0040), __byte_perm(b[4 * k + 2], b[4 * k + 3], 0x0040), 0x5410);
-        *reinterpret_cast<uint4 *>(rowg + 32 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4 *>(rowg + 32 * q + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-    }
-};
-
-template <> struct Chunk<4> {
-    __device__ __forceinline__ static void unpack(const uint8_t *rowp, int q, float2 z[16])
-    {
-        const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 16 * q);
-        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-        const float2 off = make_float2(-8388616.0f, -8388616.0f);  // -(2^23 + 8)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t x = w[k] ^ 0x88888888u;
-            const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                z[4 * k + t] = fadd2(make_float2(f_of(__byte_perm(lo, 0x4B000000u, 0x7650 + t)),
-                                                 f_of(__byte_perm(hi, 0x4B000000u, 0x7650 + t))), off);
-        }
-    }
-    __device__ __forceinline__ static void store(uint8_t *rowg, int q, const uint32_t b[32])
-    {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            uint32_t acc = b[8 * k];
-#pragma unroll
-            for (int t = 1; t < 8; ++t) acc += b[8 * k + t] << (4 * t);
-            w[k] = (acc - 0xFB000000u) ^ 0x88888888u;
-        }
-        *reinterpret_cast<uint4 *>(rowg + 16 * q) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-};
-
-template <> struct Chunk<6> {
-    __device__ __forceinline__ static void group(uint32_t lo, uint32_t hi, float2 z[4])
-    {
-        const float2 off = make_float2(-8388640.0f, -8388640.0f);  // -(2^23 + 32)
-        z[0] = fadd2(make_float2(f_of(Codec<6>::field(lo)), f_of(Codec<6>::field(lo >> 6))), off);
-        z[1] = fadd2(make_float2(f_of(Codec<6>::field(lo >> 12)), f_of(Codec<6>::field(lo >> 18))), off);
-        z[2] = fadd2(make_float2(f_of(Codec<6>::field(lo >> 24)), f_of(Codec<6>::field(__funnelshift_r(lo, hi, 30)))), off);
-        z[3] = fadd2(make_float2(f_of(Codec<6>::field(hi >> 4)), f_of(Codec<6>::field(hi >> 10))), off);
-    }
-    __device__ __forceinline__ static void unpack(const uint8_t *rowp, int q, float2 z[16])
-    {
-        const uint2 a = *reinterpret_cast<const uint2 *>(rowp + 24 * q);
-        const uint2 b = *reinterpret_cast<const uint2 *>(rowp + 24 * q + 8);
-        const uint2 c = *reinterpret_cast<const uint2 *>(rowp + 24 * q + 16);
-        group(a.x, a.y, z);
-        group(__funnelshift_r(a.y, b.x, 16), b.x >> 16, z + 4);
-        group(b.y, c.x, z + 8);
-        group(__funnelshift_r(c.x, c.y, 16), c.y >> 16, z + 12);
-    }
-    // 8 codes (b[t] = 0x4B000000 + u_t) -> 48 bits: lo (32) and hi (low 16 of the result)
-    __device__ __forceinline__ static void pack8(const uint32_t *b, uint32_t &lo, uint32_t &hi)
-    {
-        lo = b[0] + (b[1] << 6) + (b[2] << 12) + (b[3] << 18) + (b[4] << 24) + (b[5] << 30);
-        lo = (lo - 0x0B000000u) ^ 0x20820820u;
-        hi = ((b[5] >> 2) + (b[6] << 4) + (b[7] << 10)) ^ 0x8208u;
-    }
-    __device__ __forceinline__ static void store(uint8_t *rowg, int q, const uint32_t b[32])
-    {
-        uint32_t l0, h0, l1, h1, l2, h2, l3, h3;
-        pack8(b, l0, h0);
-        pack8(b + 8, l1, h1);
-        pack8(b + 16, l2, h2);
-        pack8(b + 24, l3, h3);
-        uint2 *dst = reinterpret_cast<uint2 *>(rowg + 24 * q);
-        dst[0] = make_uint2(l0, __byte_perm(h0, l1, 0x5410));
-        dst[1] = make_uint2(__byte_perm(l1, h1, 0x5432), l2);
-        dst[2] = make_uint2(__byte_perm(h2, l3, 0x5410), __byte_perm(l3, h3, 0x5432));
-    }
-};
-
 // ---------------------------------------------------------------- one tile
 //
-// Pass 1: thread (rg, cg) = (2 warp + lane / 16, lane % 16) reads rows
-// [8 rg, 8 rg + 8) x columns [8 cg, 8 cg + 8), accumulates the two column
-// sums and leaves per-warp partials in red.  B = 4, 6, 8: every row has B
+// Thread (rg, cg) = (2 warp + lane / 16, lane % 16) owns rows [8 rg, 8 rg + 8)
+// and columns [8 cg, 8 cg + 8); z[ii][p] holds columns 8 cg + 2 p, + 1 of row
+// 8 rg + ii in registers across both passes: first the old codes, then the
+// updated row values w.
+//
+// Pass 1: unpack the old codes, accumulate the two column sums and leave
+// per-warp partials in red.  B = 4, 6, 8: every row has B
 // bits (GDN); B = 0: per-row widths (KDA).
 template <int B>
-__device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R)
+__device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -416,22 +380,21 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
-        float2 z[4];
-        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + kScaleBytes + 16 * B * i, cg, z);
-        else unpack_any(R.bits[i], S.page + R.off[i], cg, z);
+        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + kScaleBytes + 16 * B * i, cg, z[ii]);
+        else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
         const float4 kl = R.kl[i];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            av[p] = ffma2(make_float2(kl.x, kl.y), z[p], av[p]);
-            ay[p] = ffma2(make_float2(kl.z, kl.w), z[p], ay[p]);
+            av[p] = ffma2(make_float2(kl.x, kl.y), z[ii][p], av[p]);
+            ay[p] = ffma2(make_float2(kl.z, kl.w), z[ii][p], ay[p]);
         }
     }
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        av[p].x += __shfl_xor_sync(0xffffffffu, av[p].x, 16);
-        av[p].y += __shfl_xor_sync(0xffffffffu, av[p].y, 16);
-        ay[p].x += __shfl_xor_sync(0xffffffffu, ay[p].x, 16);
-        ay[p].y += __shfl_xor_sync(0xffffffffu, ay[p].y, 16);
+        av[p] = fadd2(av[p], make_float2(__shfl_xor_sync(0xffffffffu, av[p].x, 16),
+                                         __shfl_xor_sync(0xffffffffu, av[p].y, 16)));
+        ay[p] = fadd2(ay[p], make_float2(__shfl_xor_sync(0xffffffffu, ay[p].x, 16),
+                                         __shfl_xor_sync(0xffffffffu, ay[p].y, 16)));
     }
     // half 0 keeps the v-sums, half 1 the y-sums; column j of a sum sits at
     // ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3) (conflict-free 16-byte stores)
@@ -504,80 +467,118 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     }
 }
 
-// Pass 2: quad q = lane % 4 of row i owns columns [32 q, 32 q + 32); each
-// thread takes rows rp and rp + 64 (rp = tid / 4).  Re-reads the old codes,
-// w = z + h u~, row absmax (local, then two shuffles), new scale, requantise,
-// store 4 b bytes of codes per row (and lane 0 the scale) to global memory.
+// Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
+// groups of the half-warp through shared memory), new scale, requantise,
+// store codes and scales to the page in global memory.
 template <int B>
-__device__ __forceinline__ void pass2_row(Smem &sm, const Stage &S, const RowCoef &R, int i, int q,
-                                          const float2 ut2[16])
-{
-    const int b = B != 0 ? B : R.bits[i];
-    const bool dropped = (R.deg[i >> 5] >> (i & 31)) & 1u;
-    const float hq = R.h[i];
-    const float2 h2 = make_float2(hq, hq);
-    float2 w[16];
-    if (!dropped) {
-        const uint8_t *rowp = S.page + (B != 0 ? kScaleBytes + 16 * B * i : R.off[i]);
-        if (B != 0) Chunk<B == 0 ? 8 : B>::unpack(rowp, q, w);
-        else if (b == 8) Chunk<8>::unpack(rowp, q, w);
-        else if (b == 6) Chunk<6>::unpack(rowp, q, w);
-        else Chunk<4>::unpack(rowp, q, w);
-#pragma unroll
-        for (int p = 0; p < 16; ++p) w[p] = ffma2(h2, ut2[p], w[p]);
-    } else {
-#pragma unroll
-        for (int p = 0; p < 16; ++p) w[p] = fmul2(h2, ut2[p]);
-    }
-    float m = fmaxf(fabsf(w[0].x), fabsf(w[0].y));
-#pragma unroll
-    for (int p = 1; p < 16; ++p) m = max3(m, fabsf(w[p].x), fabsf(w[p].y));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    const float qb = static_cast<float>((1 << (b - 1)) - 1);
-    const float mrq = R.mrq[i];
-    float inv = 0.0f, snew = 0.0f;
-    if (m >= 1e-30f && m <= 3.0e38f) {
-        inv = copysignf(qb * rcp_approx(m), mrq);
-        snew = fabsf(mrq) * m;
-    } else if (m > 0.0f && m < 1e-30f) {
-        inv = copysignf(__fdiv_rn(qb, m), mrq);
-        snew = fabsf(mrq) * m;
-    } else if (!(m == 0.0f)) {
-        atomicOr(&sm.flags, kErrNonFinite);
-    }
-    uint8_t *page = R.page;
-    if (q == 0) reinterpret_cast<float *>(page)[i] = snew;
-    const float mg = B != 0 ? Codec<B == 0 ? 8 : B>::kMagicOut : magic_out(b);
-    const float2 inv2 = make_float2(inv, inv), mg2 = make_float2(mg, mg);
-    uint32_t bits[32];
-#pragma unroll
-    for (int p = 0; p < 16; ++p) {
-        const float2 t = ffma2(w[p], inv2, mg2);
-        bits[2 * p] = __float_as_uint(t.x);
-        bits[2 * p + 1] = __float_as_uint(t.y);
-    }
-    uint8_t *rowg = page + (B != 0 ? kScaleBytes + 16 * B * i : R.off[i]);
-    if (B != 0) Chunk<B == 0 ? 8 : B>::store(rowg, q, bits);
-    else if (b == 8) Chunk<8>::store(rowg, q, bits);
-    else if (b == 6) Chunk<6>::store(rowg, q, bits);
-    else Chunk<4>::store(rowg, q, bits);
-}
-
-template <int B>
-__device__ __forceinline__ void pass2(Smem &sm, const Stage &S, const RowCoef &R)
+__device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
-    const int q = tid & 3, rp = tid >> 2;
-    float2 ut2[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float4 a = *reinterpret_cast<const float4 *>(&sm.ut[32 * q + 4 * k]);
-        ut2[2 * k] = make_float2(a.x, a.y);
-        ut2[2 * k + 1] = make_float2(a.z, a.w);
+    const int warp = tid >> 5, lane = tid & 31;
+    const int rgl = lane >> 4, cg = lane & 15;
+    const int i0 = (warp * 2 + rgl) * 8;
+    float2 ut2[4];
+    {
+        const float4 a = *reinterpret_cast<const float4 *>(&sm.ut[cg * 8]);
+        const float4 b = *reinterpret_cast<const float4 *>(&sm.ut[cg * 8 + 4]);
+        ut2[0] = make_float2(a.x, a.y);
+        ut2[1] = make_float2(a.z, a.w);
+        ut2[2] = make_float2(b.x, b.y);
+        ut2[3] = make_float2(b.z, b.w);
     }
-    pass2_row<B>(sm, S, R, rp, q, ut2);
-    pass2_row<B>(sm, S, R, rp + 64, q, ut2);
+    const uint32_t deg = (R.deg[i0 >> 5] >> (i0 & 31)) & 0xFFu;
+    float hs[8];
+    {
+        const float4 ha = *reinterpret_cast<const float4 *>(&R.h[i0]);
+        const float4 hb = *reinterpret_cast<const float4 *>(&R.h[i0 + 4]);
+        hs[0] = ha.x; hs[1] = ha.y; hs[2] = ha.z; hs[3] = ha.w;
+        hs[4] = hb.x; hs[5] = hb.y; hs[6] = hb.z; hs[7] = hb.w;
+    }
+    if (deg == 0) {
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) {
+            const float2 h2 = make_float2(hs[ii], hs[ii]);
+#pragma unroll
+            for (int p = 0; p < 4; ++p) z[ii][p] = ffma2(h2, ut2[p], z[ii][p]);
+        }
+    } else {
+#pragma unroll
+        for (int ii = 0; ii < 8; ++ii) {
+            const float2 h2 = make_float2(hs[ii], hs[ii]);
+            if (!((deg >> ii) & 1u)) {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) z[ii][p] = ffma2(h2, ut2[p], z[ii][p]);
+            } else {
+#pragma unroll
+                for (int p = 0; p < 4; ++p) z[ii][p] = fmul2(h2, ut2[p]);
+            }
+        }
+    }
+    float mx[8];
+#pragma unroll
+    for (int ii = 0; ii < 8; ++ii) {
+        float m = max3(fabsf(z[ii][0].x), fabsf(z[ii][0].y), fabsf(z[ii][1].x));
+        m = max3(m, fabsf(z[ii][1].y), fabsf(z[ii][2].x));
+        m = max3(m, fabsf(z[ii][2].y), fabsf(z[ii][3].x));
+        mx[ii] = fmaxf(m, fabsf(z[ii][3].y));
+    }
+    // row maxima: this thread's 8 partials -> shared; lane (rgl, cg) then reduces row
+    // 8 rg + (cg & 7) over the 8 column groups of half cg >> 3 (conflict-free layout)
+    float *rm = &sm.red[warp * 256];
+    {
+        float4 *dst = reinterpret_cast<float4 *>(&rm[(cg & 7) * 32 + rgl * 16 + (cg >> 3) * 8]);
+        dst[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
+        dst[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
+    }
+    __syncwarp();
+    uint8_t *page = R.page;
+    {
+        const int ii = cg & 7, half = cg >> 3;
+        const float *src = &rm[rgl * 16 + half * 8 + ii];
+        float m = max3(src[0], src[32], src[64]);
+        m = max3(m, src[96], src[128]);
+        m = max3(m, src[160], src[192]);
+        m = fmaxf(m, src[224]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        if (half == 0) {
+            const int i = i0 + ii;
+            const int b = B != 0 ? B : R.bits[i];
+            const float qb = static_cast<float>((1 << (b - 1)) - 1);
+            const float mrq = R.mrq[i];
+            float inv = 0.0f, snew = 0.0f;
+            if (m >= 1e-30f && m <= 3.0e38f) {
+                inv = copysignf(qb * rcp_approx(m), mrq);
+                snew = fabsf(mrq) * m;
+            } else if (m > 0.0f && m < 1e-30f) {
+                inv = copysignf(__fdiv_rn(qb, m), mrq);
+                snew = fabsf(mrq) * m;
+            } else if (!(m == 0.0f)) {
+                atomicOr(&sm.flags, kErrNonFinite);
+            }
+            sm.rowinv[i] = inv;
+            reinterpret_cast<float *>(page)[i] = snew;
+        }
+    }
+    __syncwarp();
+    const float4 ia = *reinterpret_cast<const float4 *>(&sm.rowinv[i0]);
+    const float4 ib = *reinterpret_cast<const float4 *>(&sm.rowinv[i0 + 4]);
+    const float invs[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+#pragma unroll
+    for (int ii = 0; ii < 8; ++ii) {
+        const int i = i0 + ii;
+        const int b = B != 0 ? B : R.bits[i];
+        const float mg = B != 0 ? Codec<B == 0 ? 8 : B>::kMagicOut : magic_out(b);
+        const float2 inv2 = make_float2(invs[ii], invs[ii]), mg2 = make_float2(mg, mg);
+        uint32_t bits[8];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 t = ffma2(z[ii][p], inv2, mg2);
+            bits[2 * p] = __float_as_uint(t.x);
+            bits[2 * p + 1] = __float_as_uint(t.y);
+        }
+        if (B != 0) Codec<B == 0 ? 8 : B>::store(page + kScaleBytes + 16 * B * i, cg, bits);
+        else store_any(b, page + R.off[i], cg, bits);
+    }
 }
 
 // ---------------------------------------------------------------- kernel
@@ -707,9 +708,9 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, const PoolView 
 //   all:       cp.async prefetch of tile i + 3's vectors, tile i + 5's location
 //   warps 0-3: column epilogue of tile i (y, u / c)
 //   warps 4-7: wait for tile i + 1's stage, its row coefficients       | barrier
-//   all:       pass 2 of tile i (re-reads the codes; new codes and scales to global memory)
-// A stage is last read by pass 2 of its tile, which every warp finishes
-// before the first barrier of the next tile.
+//   all:       pass 2 of tile i (codes held in registers; new codes and scales to global memory)
+// A stage is last read before the second barrier of its tile; thread 0
+// refills it after the first barrier of the tile after next.
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
@@ -757,11 +758,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         const Stage &S = sm.st[s];
         const bool valid = R.valid != 0;
         const int b = valid ? R.bits[0] : 8;
+        float2 z[8][4];
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0>(sm, S, R);
-            else if (b == 8) pass1<8>(sm, S, R);
-            else if (b == 6) pass1<6>(sm, S, R);
-            else pass1<4>(sm, S, R);
+            if (KIND == STQ_KDA) pass1<0>(sm, S, R, z);
+            else if (b == 8) pass1<8>(sm, S, R, z);
+            else if (b == 6) pass1<6>(sm, S, R, z);
+            else pass1<4>(sm, S, R, z);
         }
         cp_async_wait<1>();
         __syncthreads();
@@ -778,10 +780,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         timed_out = __syncthreads_or(tout) != 0;
         if (valid) {
-            if (KIND == STQ_KDA) pass2<0>(sm, S, R);
-            else if (b == 8) pass2<8>(sm, S, R);
-            else if (b == 6) pass2<6>(sm, S, R);
-            else pass2<4>(sm, S, R);
+            if (KIND == STQ_KDA) pass2<0>(sm, R, z);
+            else if (b == 8) pass2<8>(sm, R, z);
+            else if (b == 6) pass2<6>(sm, R, z);
+            else pass2<4>(sm, R, z);
         }
     }
     cp_async_wait<0>();  // no copy may land in this CTA's shared memory after it exits
