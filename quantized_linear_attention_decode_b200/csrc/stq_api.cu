@@ -255,8 +255,14 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
         uint8_t *blk = &img[o_blk + (size_t)h * stq::kHeadBlock];
         std::memcpy(blk, fr + (size_t)h * kD, kD * 4);
         std::memcpy(blk + 512, fc + (size_t)h * kD, kD * 4);
-        std::memcpy(blk + 1024, &img[o_ro + (size_t)h * kD * 2], kD * 2);
-        std::memcpy(blk + 1280, &rb[(size_t)h * kD], kD);
+        float inv_rq[kD];  // 1 / (r_i q_b(i)), rounded once from double
+        for (int i = 0; i < kD; ++i) {
+            const int b = rb[(size_t)h * kD + i];
+            inv_rq[i] = (float)(1.0 / ((double)fr[(size_t)h * kD + i] * (double)((1 << (b - 1)) - 1)));
+        }
+        std::memcpy(blk + 1024, inv_rq, kD * 4);
+        std::memcpy(blk + 1536, &img[o_ro + (size_t)h * kD * 2], kD * 2);
+        std::memcpy(blk + 1792, &rb[(size_t)h * kD], kD);
     }
 
     cudaError_t e = cudaGetDevice(&p->device);

@@ -40,9 +40,10 @@ struct __align__(128) Stage {
     uint8_t page[kMaxPage];
     // the head's table block, one bulk copy (same layout as the pool's block)
     float r[kD], c[kD];
+    float inv_rq[kD];  // 1 / (r_i q_b(i))
     uint16_t row_off[kD];
     uint8_t row_bits[kD];
-    uint8_t pad[kHeadBlock - 4 * kD - 4 * kD - 2 * kD - kD];
+    uint8_t pad[kHeadBlock - 3 * 4 * kD - 2 * kD - kD];
     // per-tile vectors, stored from registers by all threads (prefetched two tiles ahead)
     float q[kD], k[kD], v[kD], g[kD];
 };
@@ -59,7 +60,7 @@ struct __align__(16) RowCoef {
     uint8_t bits[kD];
     uint32_t deg[4];   // bit i: row i's old content is dropped (e_i = 0)
     uint8_t *page;     // the tile's page in global memory
-    float kq;
+    float kqp[4];      // k.q, partial sums of rows [32 w, 32 w + 32)
     uint32_t valid;
 };
 
@@ -72,7 +73,7 @@ struct __align__(128) Smem {
     uint8_t *stage_page[kStages];
     uint32_t stage_valid[kStages];
     float beta[kStages], alpha[kStages];
-    uint32_t raw[8][4];  // {req, slot, head offset, page bytes} of tile k in raw[k % 8]
+    uint32_t raw[8][5];  // {req, slot, head offset, page bytes, head} of tile k in raw[k % 8]
     uint32_t flags;
     unsigned long long full[kStages];
 };
@@ -418,7 +419,8 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     }
     const float cj = S.c[j];
     const float u = beta * (S.v[j] - cj * vz);
-    const float yj = fmaf(u, R.kq, cj * yz);
+    const float kq = (R.kqp[0] + R.kqp[1]) + (R.kqp[2] + R.kqp[3]);
+    const float yj = fmaf(u, kq, cj * yz);
     io.y[static_cast<size_t>(tile) * kD + j] = yj;
     sm.ut[j] = u * rcp_approx(cj);
     if (!isfinite(u) || !isfinite(yj)) atomicOr(&sm.flags, kErrNonFinite);
@@ -444,27 +446,18 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     const float ka = kr * e, la = S.q[r] * e;
     const float hq = kr * rcp_approx(e);
     const bool dropped = !(e != 0.0f && fabsf(hq) <= 1e30f);
-    const int b = S.row_bits[r];
-    const float rq = rr * static_cast<float>((1 << (b - 1)) - 1);
     R.kl[r] = make_float4(ka, ka, la, la);
     R.h[r] = dropped ? kr : hq;
-    R.mrq[r] = __fdiv_rn(dropped ? 1.0f : e, rq);
+    R.mrq[r] = (dropped ? 1.0f : e) * S.inv_rq[r];
     R.off[r] = S.row_off[r];
-    R.bits[r] = static_cast<uint8_t>(b);
+    R.bits[r] = S.row_bits[r];
     const uint32_t bal = __ballot_sync(0xffffffffu, dropped);
     if ((r & 31) == 0) R.deg[r >> 5] = bal;
     if (!isfinite(e)) atomicOr(&sm.flags, kErrNonFinite);
-    if (r < 32) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(&S.k[r * 4]);
-        const float4 q4 = *reinterpret_cast<const float4 *>(&S.q[r * 4]);
-        float a = k4.x * q4.x;
-        a = fmaf(k4.y, q4.y, a);
-        a = fmaf(k4.z, q4.z, a);
-        a = fmaf(k4.w, q4.w, a);
+    float a = kr * S.q[r];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-        if (r == 0) R.kq = a;
-    }
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if ((r & 31) == 0) R.kqp[r >> 5] = a;
 }
 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
@@ -638,10 +631,11 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
 // the first barrier of tile i, waited with wait_group 1 before the first
 // barrier of tile i + 2): q, k, v (and the KDA decay), beta, alpha of tile
 // i + 3 into its stage, and the raw location {req, slot, head offset, page
-// bytes} of tile i + 5.
+// bytes} of tile i + 5 = (request entry n5, head h5).  The small copies are
+// spread over warps 5-7, which have the least other work at this point.
 template <int KIND>
 __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const DecodeIO &io, int i, int t3, int t5,
-                                         int tiles)
+                                         int n5, int h5, int tiles)
 {
     const int t = threadIdx.x;
     if (t3 < tiles) {
@@ -652,19 +646,20 @@ __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const Deco
         else if (t < 96) cp_async16(&S.v[4 * (t - 64)], io.v + base);
         else if (t < 128) {
             if (KIND == STQ_KDA) cp_async16(&S.g[4 * (t - 96)], io.gate + base);
-        } else if (t == 128) {
+        } else if (t == 160) {
             cp_async4(&sm.beta[(i + 3) % kStages], io.beta + t3);
-        } else if (t == 129) {
+        } else if (t == 192) {
             if (KIND == STQ_GDN) cp_async4(&sm.alpha[(i + 3) % kStages], io.gate + t3);
         }
     }
-    if (t5 < tiles && t >= 130 && t < 134) {
-        const int ni = t5 / p.H, h = t5 - ni * p.H;
-        uint32_t *dst = &sm.raw[(i + 5) & 7][t - 130];
-        if (t == 130) cp_async4(dst, io.req_idx + ni);
-        else if (t == 131) cp_async4(dst, io.slot_idx + ni);
-        else if (t == 132) cp_async4(dst, p.t.head_off + h);
-        else cp_async4(dst, p.t.page_bytes + h);
+    if (t5 < tiles && t >= 224 && t < 228) {
+        uint32_t *dst = &sm.raw[(i + 5) & 7][t - 224];
+        const void *src = t == 224 ? static_cast<const void *>(io.req_idx + n5)
+                        : t == 225 ? static_cast<const void *>(io.slot_idx + n5)
+                        : t == 226 ? static_cast<const void *>(p.t.head_off + h5)
+                                   : static_cast<const void *>(p.t.page_bytes + h5);
+        cp_async4(dst, src);
+        if (t == 224) dst[4] = static_cast<uint32_t>(h5);
     }
     cp_async_commit();
 }
@@ -689,11 +684,10 @@ __device__ __forceinline__ void fill_sync(Smem &sm, const DecodeIO &io, int s, i
     }
 }
 
-__device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, const PoolView &p, int tile, int k)
+__device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
 {
     TileRaw r;
-    const int ni = tile / p.H;
-    r.h = tile - ni * p.H;
+    r.h = static_cast<int>(sm.raw[k & 7][4]);
     r.req = static_cast<int>(sm.raw[k & 7][0]);
     r.slot = static_cast<int>(sm.raw[k & 7][1]);
     r.hoff = sm.raw[k & 7][2];
@@ -704,13 +698,14 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, const PoolView 
 // Persistent CTA: tiles first, first + G, first + 2G, ... (G = gridDim.x).
 // Per tile i (stage i % 4, row data rc[i % 2]):
 //   all:       pass 1 of tile i                                        | barrier
-//   thread 0:  issue tile i + 3 (page and head block) into the stage of tile i - 1
+//   thread 96: issue tile i + 3 (page and head block) into the stage of tile i - 1
 //   all:       cp.async prefetch of tile i + 3's vectors, tile i + 5's location
 //   warps 0-3: column epilogue of tile i (y, u / c)
 //   warps 4-7: wait for tile i + 1's stage, its row coefficients       | barrier
 //   all:       pass 2 of tile i (codes held in registers; new codes and scales to global memory)
-// A stage is last read before the second barrier of its tile; thread 0
-// refills it after the first barrier of the tile after next.
+// A stage is last read before the second barrier of its tile (pass 2 reads
+// only registers and the row data); thread 96 refills it after the first
+// barrier of the next tile.
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
@@ -738,6 +733,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
                 sm.raw[a][1] = static_cast<uint32_t>(r.slot);
                 sm.raw[a][2] = r.hoff;
                 sm.raw[a][3] = r.bytes;
+                sm.raw[a][4] = static_cast<uint32_t>(r.h);
             }
         }
     }
@@ -746,11 +742,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
     __syncthreads();
     bool timed_out = false;
     if (tid >= kD) {
-        if (mbar_wait_bounded(&sm.full[0], 0)) row_setup<KIND>(sm, sm.st[0], sm.rc[0], 0);
+        // warp-uniform outcome: row_setup's shuffles need every lane
+        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND>(sm, sm.st[0], sm.rc[0], 0);
         else timed_out = true;
     }
     timed_out = __syncthreads_or(timed_out) != 0;
 
+    // (request entry, head) of tile first + 5 G, advanced by G per tile without a division
+    const int gq = G / p.H, gr = G - gq * p.H;
+    int n5 = (first + 5 * G) / p.H;
+    int h5 = first + 5 * G - n5 * p.H;
     int i = 0;
     for (int tile = first; tile < tiles && !timed_out; tile += G, ++i) {
         const int s = i % kStages;
@@ -767,16 +768,24 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         cp_async_wait<1>();
         __syncthreads();
-        if (tid == 0 && tile + 3 * G < tiles)
-            issue<KIND>(sm, (i + 3) % kStages, p, resolve(p, raw_from_smem(sm, p, tile + 3 * G, i + 3)));
-        prefetch<KIND>(sm, p, io, i, tile + 3 * G, tile + 5 * G, tiles);
+        if (tid == 96 && tile + 3 * G < tiles)  // warp 3: no vector prefetch for GDN
+            issue<KIND>(sm, (i + 3) % kStages, p, resolve(p, raw_from_smem(sm, i + 3)));
+        prefetch<KIND>(sm, p, io, i, tile + 3 * G, tile + 5 * G, n5, h5, tiles);
+        n5 += gq;
+        h5 += gr;
+        if (h5 >= p.H) {
+            h5 -= p.H;
+            ++n5;
+        }
         bool tout = false;
         if (tid < kD) {
             if (valid) column_epilogue(sm, S, R, io, tile, sm.beta[s]);
         } else if (tile + G < tiles) {
             const int sn = (i + 1) % kStages;
-            if (mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)) row_setup<KIND>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
-            else tout = true;
+            if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)))
+                row_setup<KIND>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
+            else
+                tout = true;
         }
         timed_out = __syncthreads_or(tout) != 0;
         if (valid) {

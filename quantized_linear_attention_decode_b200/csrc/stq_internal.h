@@ -25,9 +25,9 @@ constexpr uint32_t kErrTimeout = 4u;
 //   row_off[H][128] byte offset of row i inside the page (scales come first)
 //   row_bits[H][128]
 //   r[H][128], c[H][128]
-//   block[H][kHeadBlock]: r, c, row_off, row_bits of one head side by side,
-//                  so that the decode kernel fetches them with one copy
-constexpr int kHeadBlock = 1536;  // 512 (r) + 512 (c) + 256 (row_off) + 128 (row_bits), padded
+//   block[H][kHeadBlock]: r, c, 1 / (r q_b), row_off, row_bits of one head
+//                  side by side, so that the decode kernel fetches them with one copy
+constexpr int kHeadBlock = 2048;  // 512 (r) + 512 (c) + 512 (1 / (r q_b)) + 256 (row_off) + 128 (row_bits), padded
 struct Tables {
     const uint32_t *head_off;
     const uint32_t *page_bytes;
