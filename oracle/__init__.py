@@ -44,6 +44,16 @@ def lib():
         P = C.c_void_p
         L.orc_page_bytes.restype = C.c_size_t
         L.orc_page_bytes.argtypes = [C.c_int, C.c_int, P]
+        L.orc_page_bytes_fmt.restype = C.c_size_t
+        L.orc_page_bytes_fmt.argtypes = [C.c_int, C.c_int, P, C.c_int]
+        L.orc_half_to_double.restype = C.c_double
+        L.orc_half_to_double.argtypes = [C.c_uint16]
+        L.orc_double_to_half.restype = C.c_uint16
+        L.orc_double_to_half.argtypes = [C.c_double]
+        L.orc_quantize_unit_fmt.argtypes = [C.c_int, C.c_int, P, P, P, C.c_int, P, P, P]
+        L.orc_dequantize_unit_fmt.argtypes = [C.c_int, C.c_int, P, P, P, C.c_int, P, P]
+        L.orc_step_unit_fmt.argtypes = [C.c_int, C.c_int, P, P, P, C.c_int, P, P, P, P, P,
+                                        C.c_float, P, P, P]
         L.orc_get_code.restype = C.c_int32
         L.orc_get_code.argtypes = [P, C.c_int, C.c_int]
         L.orc_put_code.restype = None
@@ -75,18 +85,38 @@ def _f64(a):
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
-def page_bytes(bits, dv: int | None = None) -> int:
+# scale formats: fp32 scales (0), IEEE binary16 scales (1).  Units whose rows
+# are all 16 or all 32 bits wide are raw (binary16 / binary32 values, no scales).
+FMT_F32, FMT_F16 = 0, 1
+
+
+def is_raw(bits) -> bool:
+    return int(np.asarray(bits).reshape(-1)[0]) in (16, 32)
+
+
+def page_bytes(bits, dv: int | None = None, fmt: int = FMT_F32) -> int:
     bits = _u8(bits)
     dv = len(bits) if dv is None else dv
-    return int(lib().orc_page_bytes(len(bits), dv, _p(bits)))
+    return int(lib().orc_page_bytes_fmt(len(bits), dv, _p(bits), int(fmt)))
 
 
-def row_offsets(bits, dv: int | None = None) -> np.ndarray:
+def row_offsets(bits, dv: int | None = None, fmt: int = FMT_F32) -> np.ndarray:
     """Byte offset of every packed row inside a page (scales come first)."""
     bits = np.asarray(bits, dtype=np.int64)
     dv = len(bits) if dv is None else dv
     sizes = dv * bits // 8
-    return 4 * len(bits) + np.concatenate([[0], np.cumsum(sizes)[:-1]])
+    sb = 0 if is_raw(bits) else (2 if fmt == FMT_F16 else 4)
+    return sb * len(bits) + np.concatenate([[0], np.cumsum(sizes)[:-1]])
+
+
+def half_to_double(h: int) -> float:
+    """The value of the binary16 bit pattern h (the oracle's own decoder)."""
+    return float(lib().orc_half_to_double(int(h)))
+
+
+def double_to_half(x: float) -> int:
+    """x rounded once to binary16, ties to even (the oracle's own encoder)."""
+    return int(lib().orc_double_to_half(float(x)))
 
 
 def get_code(row: np.ndarray, b: int, j: int) -> int:
@@ -99,45 +129,48 @@ def put_code(row: np.ndarray, b: int, j: int, z: int) -> None:
     lib().orc_put_code(_p(row), b, j, int(z))
 
 
-def quantize_unit(bits, r, c, S, *, with_quot: bool = False):
+def quantize_unit(bits, r, c, S, *, with_quot: bool = False, fmt: int = FMT_F32):
     """fp32 state [dk, dv] -> packed page (uint8).  Optionally the fp32
     quotients mu / s the codes were rounded from."""
     bits, r, c, S = _u8(bits), _f32(r), _f32(c), _f32(S)
     dk, dv = S.shape
-    page = np.zeros(page_bytes(bits, dv), np.uint8)
+    page = np.zeros(page_bytes(bits, dv, fmt), np.uint8)
     quot = np.zeros((dk, dv), np.float32) if with_quot else None
-    st = lib().orc_quantize_unit(dk, dv, _p(bits), _p(r), _p(c), _p(S), _p(page), _p(quot))
+    st = lib().orc_quantize_unit_fmt(dk, dv, _p(bits), _p(r), _p(c), int(fmt), _p(S), _p(page),
+                                     _p(quot))
     if st == BADARG:
         raise ValueError("bad bit widths")
     return (page, quot, st) if with_quot else page
 
 
-def dequantize_unit(bits, r, c, page, dv: int | None = None) -> np.ndarray:
+def dequantize_unit(bits, r, c, page, dv: int | None = None, fmt: int = FMT_F32) -> np.ndarray:
     bits, r, c, page = _u8(bits), _f32(r), _f32(c), _u8(page)
     dk = len(bits)
     dv = dk if dv is None else dv
     S = np.zeros((dk, dv), np.float32)
-    st = lib().orc_dequantize_unit(dk, dv, _p(bits), _p(r), _p(c), _p(page), _p(S))
+    st = lib().orc_dequantize_unit_fmt(dk, dv, _p(bits), _p(r), _p(c), int(fmt), _p(page), _p(S))
     if st == BADARG:
         raise ValueError("bad bit widths")
     return S
 
 
-def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None):
+def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None, fmt: int = FMT_F32):
     """One quantized decode step of one unit.
 
-    Returns (page_out uint8, y float64 [dv], quot float32 [dk, dv], status)."""
+    Returns (page_out uint8, y float64 [dv], quot float32 [dk, dv], status).
+    For a raw unit quot holds fl32(X), the value before its rounding on store."""
     bits, r, c, page_in = _u8(bits), _f32(r), _f32(c), _u8(page_in)
     q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
     dk = len(bits)
     dv = len(v) if dv is None else dv
     if g.size == 1:
         g = np.full(dk, g.reshape(()), np.float32)
-    page_out = np.zeros(page_bytes(bits, dv), np.uint8)
+    page_out = np.zeros(page_bytes(bits, dv, fmt), np.uint8)
     y = np.zeros(dv, np.float64)
     quot = np.zeros((dk, dv), np.float32)
-    st = lib().orc_step_unit(dk, dv, _p(bits), _p(r), _p(c), _p(page_in), _p(page_out), _p(q),
-                             _p(k), _p(v), float(beta), _p(g), _p(y), _p(quot))
+    st = lib().orc_step_unit_fmt(dk, dv, _p(bits), _p(r), _p(c), int(fmt), _p(page_in),
+                                 _p(page_out), _p(q), _p(k), _p(v), float(beta), _p(g), _p(y),
+                                 _p(quot))
     if st == BADARG:
         raise ValueError("bad bit widths")
     return page_out, y, quot, st

@@ -32,7 +32,14 @@
  *     a_i = max_j |X_ij / (r_i c_j)| (absmax; the row factor and column
  *     factor are frozen per-head tables);
  *   - round() is IEEE round-half-to-even; the code -2^(b-1) is never made;
- *   - scales are stored as fp32;
+ *   - scales are stored as fp32 (format 0); format 1 stores them as IEEE
+ *     binary16, s16 = half(a_i / q_b) rounded to nearest even, and the codes
+ *     are then rounded from mu_ij / s16 so that s16 z reconstructs them; a
+ *     scale above the binary16 range is reported like a non-finite row;
+ *   - raw units ("FP16 pivot units" and the fp32 control state): every row
+ *     of the unit is 16 or 32 bits wide and holds the state value itself in
+ *     IEEE binary16 / binary32, with no scale and no r, c factors; the step is
+ *     the same recurrence, and X is rounded once (to nearest even) on store;
  *   - the continuous part (reconstruction, decay, retrieval, write,
  *     readout) is computed in fp64; the quantisation decision is taken in
  *     fp32 on the fp32-rounded value mu_ij = fl32(X_ij / (r_i c_j)), with
@@ -40,7 +47,9 @@
  *   - an all-zero row has s_i = 0 and all codes 0.
  *
  * Packed page of one (request, slot, head) unit, dk rows of dv codes:
- *   bytes [0, 4 dk)        fp32 scales s_0 .. s_{dk-1} (little-endian)
+ *   bytes [0, 4 dk)        fp32 scales s_0 .. s_{dk-1} (little-endian);
+ *                          [0, 2 dk) binary16 scales in format 1; no scale
+ *                          section in a raw unit
  *   then row i = 0..dk-1   dv codes of b_i bits each, dv * b_i / 8 bytes;
  *                          code j occupies bits [j b_i, (j + 1) b_i) of the
  *                          row's little-endian bit string (bit p is bit p%8
@@ -63,28 +72,88 @@ static int q_of_bits(int b) { return (1 << (b - 1)) - 1; }
 
 static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8u; }
 
+/* 16 or 32 for a raw unit (its first row decides; bits_ok checks the rest), else 0 */
+static int raw_width(int dk, const uint8_t *bits)
+{
+    if (dk <= 0) return 0;
+    return (bits[0] == 16 || bits[0] == 32) ? bits[0] : 0;
+}
+
+/* quantized rows are 4, 6 or 8 bits; a raw unit has all rows at 16 or at 32 */
 static int bits_ok(int dk, int dv, const uint8_t *bits)
 {
+    int raw = raw_width(dk, bits);
     for (int i = 0; i < dk; ++i) {
         int b = bits[i];
-        if (b != 4 && b != 6 && b != 8) return 0;
+        if (raw) {
+            if (b != raw) return 0;
+        } else if (b != 4 && b != 6 && b != 8) {
+            return 0;
+        }
         if ((dv * b) % 8 != 0) return 0;
     }
     return 1;
 }
 
-size_t orc_page_bytes(int dk, int dv, const uint8_t *bits)
+/* bytes per scale: fmt 0 fp32, fmt 1 binary16; a raw unit has none */
+static size_t scale_bytes(int dk, const uint8_t *bits, int fmt)
 {
-    size_t n = 4u * (size_t)dk;
+    if (raw_width(dk, bits)) return 0;
+    return fmt == 1 ? 2u : 4u;
+}
+
+size_t orc_page_bytes_fmt(int dk, int dv, const uint8_t *bits, int fmt)
+{
+    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk;
     for (int i = 0; i < dk; ++i) n += row_bytes(dv, bits[i]);
     return (n + 127u) / 128u * 128u;
 }
 
-static size_t row_offset(int dk, int dv, const uint8_t *bits, int i)
+size_t orc_page_bytes(int dk, int dv, const uint8_t *bits) { return orc_page_bytes_fmt(dk, dv, bits, 0); }
+
+static size_t row_offset(int dk, int dv, const uint8_t *bits, int fmt, int i)
 {
-    size_t n = 4u * (size_t)dk;
+    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk;
     for (int t = 0; t < i; ++t) n += row_bytes(dv, bits[t]);
     return n;
+}
+
+/*
+ * IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
+ * bits; exponent 0 holds zero and the subnormals f 2^-24, exponent 31 the
+ * infinities and NaNs.
+ */
+double orc_half_to_double(uint16_t h)
+{
+    int sign = h >> 15, e = (h >> 10) & 31, f = h & 1023;
+    double v;
+    if (e == 0) v = ldexp((double)f, -24);
+    else if (e == 31) v = f ? NAN : INFINITY;
+    else v = ldexp((double)(1024 + f), e - 25);
+    return sign ? -v : v;
+}
+
+/* x rounded once to the nearest binary16, ties to even (rint under the default rounding mode) */
+uint16_t orc_double_to_half(double x)
+{
+    if (isnan(x)) return 0x7E00u;
+    uint16_t sign = signbit(x) ? 0x8000u : 0u;
+    double a = fabs(x);
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: a multiple of 2^-24; 1024 units carry into the smallest normal */
+        double n = rint(ldexp(a, 24));
+        return (uint16_t)(sign | (uint16_t)n);
+    }
+    int e;
+    double m = frexp(a, &e); /* a = m 2^e, m in [0.5, 1) */
+    double t = rint(ldexp(m, 11)); /* 11 significant bits, in [1024, 2048] */
+    if (t == 2048.0) {
+        t = 1024.0;
+        e += 1;
+    }
+    int be = e - 1 + 15; /* biased exponent of t 2^(e - 11) = (t / 1024) 2^(e - 1) */
+    if (be >= 31) return (uint16_t)(sign | 0x7C00u);
+    return (uint16_t)(sign | (uint16_t)(be << 10) | (uint16_t)((int)t - 1024));
 }
 
 /* code j of a packed row, read one bit at a time, then sign-extended */
@@ -109,26 +178,72 @@ static void put_code(uint8_t *row, int b, int j, int32_t z)
     }
 }
 
-static float get_scale(const uint8_t *page, int i)
+static float get_scale(const uint8_t *page, int fmt, int i)
 {
+    if (fmt == 1) {
+        uint16_t h;
+        memcpy(&h, page + 2 * (size_t)i, 2);
+        return (float)orc_half_to_double(h);
+    }
     float s;
     memcpy(&s, page + 4 * (size_t)i, 4);
     return s;
 }
 
-static void put_scale(uint8_t *page, int i, float s) { memcpy(page + 4 * (size_t)i, &s, 4); }
+/* stores s (format 0) or half(s) (format 1); returns the value stored, as a float */
+static float put_scale(uint8_t *page, int fmt, int i, float s)
+{
+    if (fmt == 1) {
+        uint16_t h = orc_double_to_half((double)s);
+        memcpy(page + 2 * (size_t)i, &h, 2);
+        return (float)orc_half_to_double(h);
+    }
+    memcpy(page + 4 * (size_t)i, &s, 4);
+    return s;
+}
+
+/* element j of a raw row of width b (16 or 32) */
+static double get_raw(const uint8_t *row, int b, int j)
+{
+    if (b == 16) {
+        uint16_t h;
+        memcpy(&h, row + 2 * (size_t)j, 2);
+        return orc_half_to_double(h);
+    }
+    float f;
+    memcpy(&f, row + 4 * (size_t)j, 4);
+    return (double)f;
+}
+
+/* stores x rounded once to the row's format; returns the stored value */
+static double put_raw(uint8_t *row, int b, int j, double x)
+{
+    if (b == 16) {
+        uint16_t h = orc_double_to_half(x);
+        memcpy(row + 2 * (size_t)j, &h, 2);
+        return orc_half_to_double(h);
+    }
+    float f = (float)x;
+    memcpy(row + 4 * (size_t)j, &f, 4);
+    return (double)f;
+}
 
 /* exported for the pack/unpack pins */
 int32_t orc_get_code(const uint8_t *row, int b, int j) { return get_code(row, b, j); }
 void orc_put_code(uint8_t *row, int b, int j, int32_t z) { put_code(row, b, j, z); }
 
-/* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 */
+/* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 (a raw unit: the stored value) */
 static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                        const uint8_t *page, double *S)
+                        int fmt, const uint8_t *page, double *S)
 {
+    int raw = raw_width(dk, bits);
     for (int i = 0; i < dk; ++i) {
-        const uint8_t *row = page + row_offset(dk, dv, bits, i);
-        double s = (double)get_scale(page, i);
+        const uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
+        if (raw) {
+            for (int j = 0; j < dv; ++j) S[(size_t)i * dv + j] = get_raw(row, raw, j);
+            continue;
+        }
+        double s = (double)get_scale(page, fmt, i);
         for (int j = 0; j < dv; ++j) {
             int32_t z = get_code(row, bits[i], j);
             S[(size_t)i * dv + j] = s * (double)r[i] * (double)c[j] * (double)z;
@@ -143,9 +258,23 @@ static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, con
  * Returns ORC_NONFINITE if a row maximum is not finite.
  */
 static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                      const double *X, uint8_t *page, float *quot)
+                      int fmt, const double *X, uint8_t *page, float *quot)
 {
     int status = ORC_OK;
+    int raw = raw_width(dk, bits);
+    if (raw) {
+        /* raw unit: X rounded once to the row format; quot receives fl32(X) */
+        for (int i = 0; i < dk; ++i) {
+            uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
+            for (int j = 0; j < dv; ++j) {
+                double x = X[(size_t)i * dv + j];
+                double st = put_raw(row, raw, j, x);
+                if (!isfinite(st)) status = ORC_NONFINITE;
+                if (quot) quot[(size_t)i * dv + j] = (float)x;
+            }
+        }
+        return status;
+    }
     float *mu = (float *)malloc(sizeof(float) * (size_t)dv);
     for (int i = 0; i < dk; ++i) {
         int qb = q_of_bits(bits[i]);
@@ -157,9 +286,9 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
             if (!(m <= a)) a = m; /* also propagates NaN */
         }
         if (!isfinite(a)) status = ORC_NONFINITE;
-        float s = a / (float)qb;
-        put_scale(page, i, s);
-        uint8_t *row = page + row_offset(dk, dv, bits, i);
+        float s = put_scale(page, fmt, i, a / (float)qb); /* the scale as stored */
+        if (!isfinite(s)) status = ORC_NONFINITE; /* also a binary16 overflow */
+        uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
         for (int j = 0; j < dv; ++j) {
             int32_t z = 0;
             float x = 0.0f;
@@ -179,29 +308,41 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
 }
 
 /* fp32 state -> packed page (the quantizer applied to a given state) */
-int orc_quantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                      const float *S, uint8_t *page, float *quot)
+int orc_quantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                          int fmt, const float *S, uint8_t *page, float *quot)
 {
-    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
-    size_t nb = orc_page_bytes(dk, dv, bits);
+    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
+    size_t nb = orc_page_bytes_fmt(dk, dv, bits, fmt);
     memset(page, 0, nb);
     double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
     for (size_t e = 0; e < (size_t)dk * dv; ++e) X[e] = (double)S[e];
-    int st = requantize(dk, dv, bits, r, c, X, page, quot);
+    int st = requantize(dk, dv, bits, r, c, fmt, X, page, quot);
     free(X);
     return st;
 }
 
-/* packed page -> fp32 reconstruction fl32(s_i r_i c_j z_ij) */
-int orc_dequantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                        const uint8_t *page, float *S)
+int orc_quantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      const float *S, uint8_t *page, float *quot)
 {
-    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
+    return orc_quantize_unit_fmt(dk, dv, bits, r, c, 0, S, page, quot);
+}
+
+/* packed page -> fp32 reconstruction fl32(s_i r_i c_j z_ij) (a raw unit: its values) */
+int orc_dequantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                            int fmt, const uint8_t *page, float *S)
+{
+    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
     double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
-    reconstruct(dk, dv, bits, r, c, page, X);
+    reconstruct(dk, dv, bits, r, c, fmt, page, X);
     for (size_t e = 0; e < (size_t)dk * dv; ++e) S[e] = (float)X[e];
     free(X);
     return ORC_OK;
+}
+
+int orc_dequantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                        const uint8_t *page, float *S)
+{
+    return orc_dequantize_unit_fmt(dk, dv, bits, r, c, 0, page, S);
 }
 
 /*
@@ -216,17 +357,17 @@ int orc_dequantize_unit(int dk, int dv, const uint8_t *bits, const float *r, con
  * y is returned in fp64; quot (optional, dk*dv floats) receives the fp32
  * quotients the new codes were rounded from.
  */
-int orc_step_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                  const uint8_t *page_in, uint8_t *page_out,
-                  const float *q, const float *k, const float *v, float beta, const float *g,
-                  double *y, float *quot)
+int orc_step_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      int fmt, const uint8_t *page_in, uint8_t *page_out,
+                      const float *q, const float *k, const float *v, float beta, const float *g,
+                      double *y, float *quot)
 {
-    if (!bits_ok(dk, dv, bits)) return ORC_BADARG;
+    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
     size_t nel = (size_t)dk * dv;
     double *P = (double *)malloc(sizeof(double) * nel);
     double *vo = (double *)malloc(sizeof(double) * (size_t)dv);
     double *u = (double *)malloc(sizeof(double) * (size_t)dv);
-    reconstruct(dk, dv, bits, r, c, page_in, P);
+    reconstruct(dk, dv, bits, r, c, fmt, page_in, P);
     for (int i = 0; i < dk; ++i)
         for (int j = 0; j < dv; ++j) P[(size_t)i * dv + j] *= (double)g[i];
     for (int j = 0; j < dv; ++j) {
@@ -242,14 +383,22 @@ int orc_step_unit(int dk, int dv, const uint8_t *bits, const float *r, const flo
         for (int i = 0; i < dk; ++i) acc += (double)q[i] * P[(size_t)i * dv + j];
         y[j] = acc;
     }
-    memset(page_out, 0, orc_page_bytes(dk, dv, bits));
-    int st = requantize(dk, dv, bits, r, c, P, page_out, quot);
+    memset(page_out, 0, orc_page_bytes_fmt(dk, dv, bits, fmt));
+    int st = requantize(dk, dv, bits, r, c, fmt, P, page_out, quot);
     for (int j = 0; j < dv; ++j)
         if (!isfinite(y[j])) st = ORC_NONFINITE;
     free(P);
     free(vo);
     free(u);
     return st;
+}
+
+int orc_step_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                  const uint8_t *page_in, uint8_t *page_out,
+                  const float *q, const float *k, const float *v, float beta, const float *g,
+                  double *y, float *quot)
+{
+    return orc_step_unit_fmt(dk, dv, bits, r, c, 0, page_in, page_out, q, k, v, beta, g, y, quot);
 }
 
 /*
