@@ -62,8 +62,15 @@ typedef struct stq_pool stq_pool;
 /*
  * Pool description ("SGLang state pool" section: pool = concurrency x slots
  * x per-request state).  A unit of precision ("core method" section: a whole
- * head for GDN, one key row for KDA) carries a bit width b in {4, 6, 8}.
+ * head for GDN, one key row for KDA) carries a bit width b in {4, 6, 8}
+ * (quantized codes).  Raw pools hold the state values themselves: every unit
+ * at 16 (IEEE binary16, the page's FP16 "pivot" storage applied to the whole
+ * pool) or every unit at 32 (fp32, the unquantized control the page's
+ * state-update timings compare against); mixing raw and quantized units in
+ * one pool returns STQ_ERR_UNSUPPORTED.
  */
+#define STQ_SCALE_F16 1u /* flags: per-row scales stored as IEEE binary16 ("method steps", step 6) */
+
 typedef struct {
     int32_t kind;         /* stq_kind */
     int32_t num_requests; /* R >= 1 */
@@ -74,11 +81,16 @@ typedef struct {
     const uint8_t *unit_bits;  /* host; GDN: [H] one width per head; KDA: [H * d_k] one per key row */
     const float *row_factor;   /* host; [H * d_k] r_i, finite and > 0; NULL means all 1 */
     const float *col_factor;   /* host; [H * d_v] c_j, finite and > 0; NULL means all 1 */
+    uint32_t flags;            /* 0 (fp32 scales) or STQ_SCALE_F16; must be 0 for a raw pool */
 } stq_pool_desc;
 
 /*
  * Packed page of one (request, slot, head) state, in device memory:
- *   bytes [0, 512)   128 fp32 scales s_i, one per key row
+ *   bytes [0, 512)   128 fp32 scales s_i, one per key row ([0, 256): 128
+ *                    binary16 scales with STQ_SCALE_F16; codes are then
+ *                    rounded from mu / s16 so that s16 z reconstructs them,
+ *                    and a scale beyond the binary16 range is reported as
+ *                    STQ_ERR_NONFINITE)
  *   then rows i = 0..127 in order, row i holding 128 codes of b_i bits
  *   (16 * b_i bytes); code j occupies bits [j b_i, (j+1) b_i) of the row's
  *   little-endian bit string, as a b_i-bit two's complement integer in
@@ -87,6 +99,9 @@ typedef struct {
  * The pages of heads 0..H-1 follow each other inside a slot; slots are
  * ordered [request][slot].  The state the page stands for is
  *   S^_ij = s_i * r_i * c_j * z_ij          ("core method": X^ = r c z).
+ * A raw page (units of 16 or 32 bits) is the row-major 128 x 128 state in
+ * binary16 or fp32 (32 KiB or 64 KiB), with no scales; r and c do not apply,
+ * and every step rounds X once (to nearest even) into it.
  */
 
 /* Allocate a pool (device memory, all states zero) for the current device. */

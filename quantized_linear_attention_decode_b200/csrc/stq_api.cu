@@ -14,6 +14,7 @@
 
 struct stq_pool {
     int kind = 0, R = 0, S = 0, H = 0;
+    int scale_bytes = 4, raw_bits = 0;
     int device = 0;
     size_t slot_bytes = 0, packed_bytes = 0;
     uint8_t *d_pages = nullptr;
@@ -51,22 +52,31 @@ bool fault(const char *which)
     return f != nullptr && std::strcmp(f, which) == 0;
 }
 
-// Layout of one head's page from its row bit widths.
+// Layout of one head's page from its row bit widths and the bytes per row
+// scale (4 fp32, 2 binary16, 0 for a raw page).
 struct HeadLayout {
     uint32_t page_bytes;
     uint16_t row_off[stq::kD];
 };
 
-HeadLayout head_layout(const uint8_t *row_bits)
+HeadLayout head_layout(const uint8_t *row_bits, int scale_bytes)
 {
     HeadLayout L{};
-    uint32_t off = stq::kScaleBytes;
+    uint32_t off = (uint32_t)scale_bytes * stq::kD;
     for (int i = 0; i < stq::kD; ++i) {
         L.row_off[i] = (uint16_t)off;
         off += 16u * row_bits[i];
     }
     L.page_bytes = (off + stq::kPageAlign - 1) / stq::kPageAlign * stq::kPageAlign;
     return L;
+}
+
+// Bytes per row scale of a (validated) description: 0 for a raw pool.
+int scale_bytes_of(const stq_pool_desc *d)
+{
+    const int b0 = d->unit_bits[0];
+    if (b0 == 16 || b0 == 32) return 0;
+    return (d->flags & STQ_SCALE_F16) ? 2 : 4;
 }
 
 // Validates a description; fills the per-row bit table [H][128].
@@ -82,11 +92,18 @@ stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
     if (d->unit_bits == nullptr) return fail(STQ_ERR_ARG, "unit_bits is NULL");
     const int H = d->num_heads;
     const size_t nunits = d->kind == STQ_GDN ? (size_t)H : (size_t)H * stq::kD;
+    if (d->flags & ~STQ_SCALE_F16) return fail(STQ_ERR_ARG, "flags 0x%x", d->flags);
+    const int b0 = d->unit_bits[0];
+    const bool raw = b0 == 16 || b0 == 32;
     for (size_t u = 0; u < nunits; ++u) {
         int b = d->unit_bits[u];
-        if (b != 4 && b != 6 && b != 8)
-            return fail(STQ_ERR_ARG, "unit_bits[%zu] = %d (must be 4, 6 or 8)", u, b);
+        if (b != 4 && b != 6 && b != 8 && b != 16 && b != 32)
+            return fail(STQ_ERR_ARG, "unit_bits[%zu] = %d (must be 4, 6, 8, 16 or 32)", u, b);
+        if (raw ? b != b0 : (b == 16 || b == 32))
+            return fail(STQ_ERR_UNSUPPORTED, "unit_bits[%zu] = %d: raw (16 / 32-bit) units must make up "
+                        "the whole pool, at one width", u, b);
     }
+    if (raw && d->flags != 0) return fail(STQ_ERR_ARG, "a raw pool has no scales (flags must be 0)");
     for (int which = 0; which < 2; ++which) {
         const float *f = which ? d->col_factor : d->row_factor;
         if (f == nullptr) continue;
@@ -110,8 +127,9 @@ stq_status sizes_of(const stq_pool_desc *d, const std::vector<uint8_t> &row_bits
                     size_t *slot_bytes, size_t *packed)
 {
     size_t off = 0;
+    const int sb = scale_bytes_of(d);
     for (int h = 0; h < d->num_heads; ++h) {
-        HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD]);
+        HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD], sb);
         if (head_off) head_off->push_back((uint32_t)off);
         if (page_bytes) page_bytes->push_back(L.page_bytes);
         off += L.page_bytes;
@@ -133,6 +151,8 @@ stq::PoolView view(stq_pool *p)
     v.S = p->S;
     v.H = p->H;
     v.kind = p->kind;
+    v.scale_bytes = p->scale_bytes;
+    v.raw_bits = p->raw_bits;
     v.t = p->t;
     v.err = p->d_err;
     return v;
@@ -223,6 +243,8 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->R = desc->num_requests;
     p->S = desc->num_slots;
     p->H = desc->num_heads;
+    p->scale_bytes = scale_bytes_of(desc);
+    p->raw_bits = p->scale_bytes == 0 ? desc->unit_bits[0] : 0;
     st = sizes_of(desc, rb, &p->head_off, &p->page_bytes, &p->slot_bytes, &p->packed_bytes);
     if (st != STQ_OK) {
         delete p;
@@ -241,7 +263,7 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     std::memcpy(&img[o_hoff], p->head_off.data(), n_hoff);
     std::memcpy(&img[o_pb], p->page_bytes.data(), n_pb);
     for (int h = 0; h < H; ++h) {
-        HeadLayout L = head_layout(&rb[(size_t)h * kD]);
+        HeadLayout L = head_layout(&rb[(size_t)h * kD], p->scale_bytes);
         std::memcpy(&img[o_ro + (size_t)h * kD * 2], L.row_off, kD * 2);
     }
     std::memcpy(&img[o_rb], rb.data(), n_rb);
@@ -255,10 +277,11 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
         uint8_t *blk = &img[o_blk + (size_t)h * stq::kHeadBlock];
         std::memcpy(blk, fr + (size_t)h * kD, kD * 4);
         std::memcpy(blk + 512, fc + (size_t)h * kD, kD * 4);
-        float inv_rq[kD];  // 1 / (r_i q_b(i)), rounded once from double
+        float inv_rq[kD];  // 1 / (r_i q_b(i)), rounded once from double (unused by raw pages)
         for (int i = 0; i < kD; ++i) {
             const int b = rb[(size_t)h * kD + i];
-            inv_rq[i] = (float)(1.0 / ((double)fr[(size_t)h * kD + i] * (double)((1 << (b - 1)) - 1)));
+            inv_rq[i] = b <= 8 ? (float)(1.0 / ((double)fr[(size_t)h * kD + i] * (double)((1 << (b - 1)) - 1)))
+                               : 0.0f;
         }
         std::memcpy(blk + 1024, inv_rq, kD * 4);
         std::memcpy(blk + 1536, &img[o_ro + (size_t)h * kD * 2], kD * 2);
@@ -377,7 +400,8 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
     DeviceGuard g(p->device);
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y};
-    cudaError_t e = stq::launch_decode(view(p), io, (cudaStream_t)stream);
+    cudaError_t e = p->raw_bits ? stq::launch_decode_raw(view(p), io, (cudaStream_t)stream)
+                                : stq::launch_decode(view(p), io, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "decode launch");
 }
 

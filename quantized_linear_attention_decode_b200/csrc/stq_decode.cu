@@ -26,6 +26,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_fp16.h>
+
 #include "stq_internal.h"
 
 namespace stq {
@@ -368,7 +370,7 @@ __device__ __forceinline__ float magic_out(int b)
 // Pass 1: unpack the old codes, accumulate the two column sums and leave
 // per-warp partials in red.  B = 4, 6, 8: every row has B
 // bits (GDN); B = 0: per-row widths (KDA).
-template <int B>
+template <int B, int SB>
 __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -381,7 +383,7 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
-        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + kScaleBytes + 16 * B * i, cg, z[ii]);
+        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + 16 * B * i, cg, z[ii]);
         else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
         const float4 kl = R.kl[i];
 #pragma unroll
@@ -428,7 +430,7 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
 
 // Per row (threads 128..255) of the next tile: decayed scale e_i and the
 // coefficients both passes need; warp 4 also forms k.q.
-template <int KIND>
+template <int KIND, int SB>
 __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, int s)
 {
     const int r = threadIdx.x - kD;
@@ -438,7 +440,8 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
         R.valid = valid;
     }
     if (!valid) return;
-    const float sc = reinterpret_cast<const float *>(S.page)[r];
+    const float sc = SB == 4 ? reinterpret_cast<const float *>(S.page)[r]
+                             : __half2float(reinterpret_cast<const __half *>(S.page)[r]);
     const float g = KIND == STQ_GDN ? sm.alpha[s] : S.g[r];
     const float rr = S.r[r];
     const float e = (g * sc) * rr;
@@ -463,7 +466,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
 // groups of the half-warp through shared memory), new scale, requantise,
 // store codes and scales to the page in global memory.
-template <int B>
+template <int B, int SB>
 __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -525,6 +528,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
     }
     __syncwarp();
     uint8_t *page = R.page;
+    bool clip = false;  // binary16 scale below a / q_b in the subnormal range: codes need clipping
     {
         const int ii = cg & 7, half = cg >> 3;
         const float *src = &rm[rgl * 16 + half * 8 + ii];
@@ -539,19 +543,36 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
             const float qb = static_cast<float>((1 << (b - 1)) - 1);
             const float mrq = R.mrq[i];
             float inv = 0.0f, snew = 0.0f;
-            if (m >= 1e-30f && m <= 3.0e38f) {
-                inv = copysignf(qb * rcp_approx(m), mrq);
-                snew = fabsf(mrq) * m;
-            } else if (m > 0.0f && m < 1e-30f) {
-                inv = copysignf(__fdiv_rn(qb, m), mrq);
-                snew = fabsf(mrq) * m;
-            } else if (!(m == 0.0f)) {
-                atomicOr(&sm.flags, kErrNonFinite);
+            if (SB == 4) {
+                if (m >= 1e-30f && m <= 3.0e38f) {
+                    inv = copysignf(qb * rcp_approx(m), mrq);
+                    snew = fabsf(mrq) * m;
+                } else if (m > 0.0f && m < 1e-30f) {
+                    inv = copysignf(__fdiv_rn(qb, m), mrq);
+                    snew = fabsf(mrq) * m;
+                } else if (!(m == 0.0f)) {
+                    atomicOr(&sm.flags, kErrNonFinite);
+                }
+                reinterpret_cast<float *>(page)[i] = snew;
+            } else {
+                // binary16 scale: s16 = half(a / q_b); the codes are rounded from
+                // mu / s16 = w (e / r) / s16 = w mrq q_b / s16
+                const float s = fabsf(mrq) * m;
+                const __half s16 = __float2half_rn(s);
+                const float sf = __half2float(s16);
+                if (sf > 0.0f && sf <= 65504.0f) inv = mrq * qb * rcp_approx(sf);
+                else if (!(sf == 0.0f)) atomicOr(&sm.flags, kErrNonFinite);  // overflow or NaN
+                // for a normal binary16 scale s / s16 <= 1 + 2^-11, so |w inv| <= q_b (1 + 2^-11)
+                // rounds to at most q_b (q_b <= 127); only a subnormal s16 can round further down
+                clip = sf < s && sf < 6.103515625e-05f;
+                reinterpret_cast<__half *>(page)[i] = s16;
             }
             sm.rowinv[i] = inv;
-            reinterpret_cast<float *>(page)[i] = snew;
         }
     }
+    // bit ii: row i0 + ii needs its codes clipped (lanes 0-7 and 16-23 decided rows of
+    // row groups 2 warp and 2 warp + 1)
+    const uint32_t clipm = SB == 2 ? (__ballot_sync(0xffffffffu, clip) >> (rgl * 16)) & 0xFFu : 0u;
     __syncwarp();
     const float4 ia = *reinterpret_cast<const float4 *>(&sm.rowinv[i0]);
     const float4 ib = *reinterpret_cast<const float4 *>(&sm.rowinv[i0 + 4]);
@@ -565,11 +586,18 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
         uint32_t bits[8];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            const float2 t = ffma2(z[ii][p], inv2, mg2);
+            float2 t = ffma2(z[ii][p], inv2, mg2);
+            if (SB == 2 && ((clipm >> ii) & 1u)) {
+                // the binary16 scale rounded below a / q_b by up to half a subnormal step:
+                // clip the rounded quotient to [-q_b, q_b]
+                const float qb = static_cast<float>((1 << (b - 1)) - 1);
+                t.x = fminf(fmaxf(t.x, mg - qb), mg + qb);
+                t.y = fminf(fmaxf(t.y, mg - qb), mg + qb);
+            }
             bits[2 * p] = __float_as_uint(t.x);
             bits[2 * p + 1] = __float_as_uint(t.y);
         }
-        if (B != 0) Codec<B == 0 ? 8 : B>::store(page + kScaleBytes + 16 * B * i, cg, bits);
+        if (B != 0) Codec<B == 0 ? 8 : B>::store(page + SB * kD + 16 * B * i, cg, bits);
         else store_any(b, page + R.off[i], cg, bits);
     }
 }
@@ -706,7 +734,7 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
 // A stage is last read before the second barrier of its tile (pass 2 reads
 // only registers and the row data); thread 96 refills it after the first
 // barrier of the next tile.
-template <int KIND>
+template <int KIND, int SB>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -743,7 +771,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
     bool timed_out = false;
     if (tid >= kD) {
         // warp-uniform outcome: row_setup's shuffles need every lane
-        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND>(sm, sm.st[0], sm.rc[0], 0);
+        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB>(sm, sm.st[0], sm.rc[0], 0);
         else timed_out = true;
     }
     timed_out = __syncthreads_or(timed_out) != 0;
@@ -761,10 +789,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         const int b = valid ? R.bits[0] : 8;
         float2 z[8][4];
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0>(sm, S, R, z);
-            else if (b == 8) pass1<8>(sm, S, R, z);
-            else if (b == 6) pass1<6>(sm, S, R, z);
-            else pass1<4>(sm, S, R, z);
+            if (KIND == STQ_KDA) pass1<0, SB>(sm, S, R, z);
+            else if (b == 8) pass1<8, SB>(sm, S, R, z);
+            else if (b == 6) pass1<6, SB>(sm, S, R, z);
+            else pass1<4, SB>(sm, S, R, z);
         }
         cp_async_wait<1>();
         __syncthreads();
@@ -783,16 +811,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         } else if (tile + G < tiles) {
             const int sn = (i + 1) % kStages;
             if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)))
-                row_setup<KIND>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
+                row_setup<KIND, SB>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
             else
                 tout = true;
         }
         timed_out = __syncthreads_or(tout) != 0;
         if (valid) {
-            if (KIND == STQ_KDA) pass2<0>(sm, R, z);
-            else if (b == 8) pass2<8>(sm, R, z);
-            else if (b == 6) pass2<6>(sm, R, z);
-            else pass2<4>(sm, R, z);
+            if (KIND == STQ_KDA) pass2<0, SB>(sm, R, z);
+            else if (b == 8) pass2<8, SB>(sm, R, z);
+            else if (b == 6) pass2<6, SB>(sm, R, z);
+            else pass2<4, SB>(sm, R, z);
         }
     }
     cp_async_wait<0>();  // no copy may land in this CTA's shared memory after it exits
@@ -814,7 +842,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
 
 constexpr int kMaxDevices = 64;
 
-template <int KIND>
+template <int KIND, int SB>
 cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
     // per device: SM count, and the dynamic shared-memory opt-in of this kernel
@@ -828,13 +856,13 @@ cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(decode_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<KIND, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         sms[dev] = n > 0 ? n : 148;
     }
     const int tiles = io.n * p.H;
     const int grid = tiles < 2 * sms[dev] ? tiles : 2 * sms[dev];
-    decode_kernel<KIND><<<grid, kThreads, smem, stream>>>(p, io, tiles);
+    decode_kernel<KIND, SB><<<grid, kThreads, smem, stream>>>(p, io, tiles);
     count_launch();
     return cudaGetLastError();
 }
@@ -843,7 +871,9 @@ cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 
 cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
-    return p.kind == STQ_KDA ? launch<STQ_KDA>(p, io, stream) : launch<STQ_GDN>(p, io, stream);
+    if (p.scale_bytes == 2)
+        return p.kind == STQ_KDA ? launch<STQ_KDA, 2>(p, io, stream) : launch<STQ_GDN, 2>(p, io, stream);
+    return p.kind == STQ_KDA ? launch<STQ_KDA, 4>(p, io, stream) : launch<STQ_GDN, 4>(p, io, stream);
 }
 
 }  // namespace stq

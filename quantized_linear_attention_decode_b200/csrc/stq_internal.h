@@ -43,6 +43,8 @@ struct PoolView {
     size_t slot_bytes;
     int R, S, H;
     int kind;
+    int scale_bytes;     // bytes per row scale: 4 (fp32) or 2 (binary16); 0 in a raw pool
+    int raw_bits;        // 16 or 32 in a raw pool (every unit), else 0
     Tables t;
     uint32_t *err;
 };
@@ -56,6 +58,7 @@ struct DecodeIO {
 };
 
 cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+cudaError_t launch_decode_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                             int n, const float *state, cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,

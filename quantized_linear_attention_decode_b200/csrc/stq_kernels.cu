@@ -6,10 +6,13 @@
 // "PTQ" (Q(x) = s clip(round(x/s), -q_b, q_b)), "core method"
 // (X^_ij = r_i c_j z_ij), "method steps" (online decode steps 1-7).
 //
-// Page layout (one (request, slot, head) tile): 128 fp32 row scales, then
-// 128 rows of 128 b_i-bit two's complement codes (16 b_i bytes per row,
-// little-endian bit order), padded to 128 bytes.
+// Page layout (one (request, slot, head) tile): 128 fp32 row scales (or 128
+// binary16 scales), then 128 rows of 128 b_i-bit two's complement codes
+// (16 b_i bytes per row, little-endian bit order), padded to 128 bytes.  A raw
+// page is the row-major state itself in binary16 or fp32.
 #include <cstdint>
+
+#include <cuda_fp16.h>
 
 #include "stq_internal.h"
 
@@ -61,7 +64,10 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-        const float s = __fdiv_rn(a, static_cast<float>(qb));
+        float s = __fdiv_rn(a, static_cast<float>(qb));
+        __half s16 = __float2half_rn(s);
+        if (p.scale_bytes == 2) s = __half2float(s16);  // the scale as stored
+        bad |= !isfinite(s);
         uint32_t code[4];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -86,7 +92,10 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
             row[lane * 3 + 1] = static_cast<uint8_t>(w >> 8);
             row[lane * 3 + 2] = static_cast<uint8_t>(w >> 16);
         }
-        if (lane == 0) reinterpret_cast<float *>(page)[i] = s;
+        if (lane == 0) {
+            if (p.scale_bytes == 2) reinterpret_cast<__half *>(page)[i] = s16;
+            else reinterpret_cast<float *>(page)[i] = s;
+        }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrNonFinite);
 }
@@ -109,8 +118,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
     const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
     for (int i = warp; i < kD; i += 8) {
         const int b = p.t.row_bits[h * kD + i];
-        const double sr = static_cast<double>(reinterpret_cast<const float *>(page)[i]) *
-                          static_cast<double>(p.t.r[h * kD + i]);
+        const float sc = p.scale_bytes == 2 ? __half2float(reinterpret_cast<const __half *>(page)[i])
+                                            : reinterpret_cast<const float *>(page)[i];
+        const double sr = static_cast<double>(sc) * static_cast<double>(p.t.r[h * kD + i]);
         const uint8_t *row = page + p.t.row_off[h * kD + i];
         int zz[4];
         if (b == 8) {
@@ -135,12 +145,75 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
     }
 }
 
+// Raw pages: the state rounded once to binary16 (round to nearest even) or
+// copied as fp32, and back.  256 threads, 4 consecutive elements each per step.
+template <int BITS>
+__global__ void __launch_bounds__(256) quantize_raw_kernel(PoolView p, const int32_t *req_idx,
+                                                           const int32_t *slot_idx, const float *state)
+{
+    const int tile = blockIdx.x;
+    const int ni = tile / p.H, h = tile - ni * p.H;
+    const int req = req_idx[ni], slot = slot_idx[ni];
+    if (req < 0 || req >= p.R || slot < 0 || slot >= p.S) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrIndex);
+        return;
+    }
+    uint8_t *page = tile_page(p, req, slot, h);
+    const float *S = state + static_cast<size_t>(tile) * kD * kD;
+    bool bad = false;
+    for (int e = threadIdx.x * 4; e < kD * kD; e += 256 * 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(S + e);
+        if (BITS == 32) {
+            *reinterpret_cast<float4 *>(page + 4 * e) = x;
+            bad |= !(isfinite(x.x) && isfinite(x.y) && isfinite(x.z) && isfinite(x.w));
+        } else {
+            const __half2 a = __floats2half2_rn(x.x, x.y), b = __floats2half2_rn(x.z, x.w);
+            uint2 w;
+            w.x = *reinterpret_cast<const uint32_t *>(&a);
+            w.y = *reinterpret_cast<const uint32_t *>(&b);
+            *reinterpret_cast<uint2 *>(page + 2 * e) = w;
+            const float2 fa = __half22float2(a), fb = __half22float2(b);
+            bad |= !(isfinite(fa.x) && isfinite(fa.y) && isfinite(fb.x) && isfinite(fb.y));
+        }
+    }
+    if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(p.err, kErrNonFinite);
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(256) dequantize_raw_kernel(PoolView p, const int32_t *req_idx,
+                                                             const int32_t *slot_idx, float *state)
+{
+    const int tile = blockIdx.x;
+    const int ni = tile / p.H, h = tile - ni * p.H;
+    const int req = req_idx[ni], slot = slot_idx[ni];
+    if (req < 0 || req >= p.R || slot < 0 || slot >= p.S) {
+        if (threadIdx.x == 0) atomicOr(p.err, kErrIndex);
+        return;
+    }
+    const uint8_t *page = tile_page(p, req, slot, h);
+    float *S = state + static_cast<size_t>(tile) * kD * kD;
+    for (int e = threadIdx.x * 4; e < kD * kD; e += 256 * 4) {
+        float4 x;
+        if (BITS == 32) {
+            x = *reinterpret_cast<const float4 *>(page + 4 * e);
+        } else {
+            const uint2 w = *reinterpret_cast<const uint2 *>(page + 2 * e);
+            const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&w.x));
+            const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&w.y));
+            x = make_float4(a.x, a.y, b.x, b.y);
+        }
+        *reinterpret_cast<float4 *>(S + e) = x;
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                             int n, const float *state, cudaStream_t stream)
 {
-    quantize_kernel<<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    if (p.raw_bits == 32) quantize_raw_kernel<32><<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    else if (p.raw_bits == 16) quantize_raw_kernel<16><<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    else quantize_kernel<<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
     count_launch();
     return cudaGetLastError();
 }
@@ -148,7 +221,9 @@ cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int
 cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                               int n, float *state, cudaStream_t stream)
 {
-    dequantize_kernel<<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    if (p.raw_bits == 32) dequantize_raw_kernel<32><<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    else if (p.raw_bits == 16) dequantize_raw_kernel<16><<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
+    else dequantize_kernel<<<n * p.H, 256, 0, stream>>>(p, req_idx, slot_idx, state);
     count_launch();
     return cudaGetLastError();
 }

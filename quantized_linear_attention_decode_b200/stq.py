@@ -15,6 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libstq.so")
 
 STQ_GDN, STQ_KDA = 0, 1
+STQ_SCALE_F16 = 1  # desc flag: per-row scales stored as IEEE binary16
 STATUS = {0: "STQ_OK", 1: "STQ_ERR_ARG", 2: "STQ_ERR_OOM", 3: "STQ_ERR_CUDA", 4: "STQ_ERR_INDEX",
           5: "STQ_ERR_NONFINITE", 6: "STQ_ERR_UNSUPPORTED", 7: "STQ_ERR_TIMEOUT"}
 STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE, \
@@ -36,7 +37,8 @@ class StqError(RuntimeError):
 class _Desc(C.Structure):
     _fields_ = [("kind", C.c_int32), ("num_requests", C.c_int32), ("num_slots", C.c_int32),
                 ("num_heads", C.c_int32), ("d_k", C.c_int32), ("d_v", C.c_int32),
-                ("unit_bits", C.c_void_p), ("row_factor", C.c_void_p), ("col_factor", C.c_void_p)]
+                ("unit_bits", C.c_void_p), ("row_factor", C.c_void_p), ("col_factor", C.c_void_p),
+                ("flags", C.c_uint32)]
 
 
 _lib = None
@@ -108,22 +110,23 @@ def _dev(t, dtype, shape=None, name="tensor"):
     return C.c_void_p(t.data_ptr())
 
 
-def _desc(kind, R, S, H, unit_bits, row_factor, col_factor, keep):
+def _desc(kind, R, S, H, unit_bits, row_factor, col_factor, keep, flags=0):
     ub = np.ascontiguousarray(unit_bits, np.uint8)
     rf = None if row_factor is None else np.ascontiguousarray(row_factor, np.float32)
     cf = None if col_factor is None else np.ascontiguousarray(col_factor, np.float32)
     keep.extend([ub, rf, cf])
     ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
-    return _Desc(int(kind), int(R), int(S), int(H), 128, 128, ptr(ub), ptr(rf), ptr(cf))
+    return _Desc(int(kind), int(R), int(S), int(H), 128, 128, ptr(ub), ptr(rf), ptr(cf), int(flags))
 
 
 class Pool:
     """Owner of one stq_pool handle (destroyed with the object)."""
 
-    def __init__(self, handle, kind, R, S, H, unit_bits):
+    def __init__(self, handle, kind, R, S, H, unit_bits, flags=0):
         self.handle = handle
         self.kind, self.R, self.S, self.H = kind, R, S, H
         self.unit_bits = np.asarray(unit_bits, np.uint8).copy()
+        self.flags = int(flags)
 
     def __del__(self):
         self.close()
@@ -149,12 +152,12 @@ class Pool:
 
 
 def stq_pool_create(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
-                    col_factor=None) -> Pool:
+                    col_factor=None, flags=0) -> Pool:
     keep = []
-    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep)
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags)
     h = C.c_void_p()
     _check(load().stq_pool_create(C.byref(d), C.byref(h)))
-    return Pool(h, kind, num_requests, num_slots, num_heads, unit_bits)
+    return Pool(h, kind, num_requests, num_slots, num_heads, unit_bits, flags)
 
 
 def stq_pool_destroy(pool: Pool) -> None:
@@ -168,9 +171,9 @@ def stq_pool_bytes(pool: Pool):
 
 
 def stq_desc_bytes(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
-                   col_factor=None):
+                   col_factor=None, flags=0):
     keep = []
-    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep)
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags)
     a, b = C.c_size_t(), C.c_size_t()
     _check(load().stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)))
     return a.value, b.value

@@ -12,27 +12,43 @@ import numpy as np
 D = 128
 
 
-def page_bytes(row_bits) -> int:
-    n = 4 * D + 16 * int(np.sum(np.asarray(row_bits, np.int64)))
+def _scale_bytes(row_bits, fmt) -> int:
+    if int(np.asarray(row_bits).reshape(-1)[0]) in (16, 32):
+        return 0  # raw page
+    return 2 if fmt == 1 else 4
+
+
+def page_bytes(row_bits, fmt: int = 0) -> int:
+    n = _scale_bytes(row_bits, fmt) * D + 16 * int(np.sum(np.asarray(row_bits, np.int64)))
     return (n + 127) // 128 * 128
 
 
-def row_offsets(row_bits) -> np.ndarray:
+def row_offsets(row_bits, fmt: int = 0) -> np.ndarray:
     rb = np.asarray(row_bits, np.int64)
-    return 4 * D + np.concatenate([[0], np.cumsum(16 * rb)[:-1]])
+    return _scale_bytes(row_bits, fmt) * D + np.concatenate([[0], np.cumsum(16 * rb)[:-1]])
 
 
-def head_offsets(pool_row_bits) -> np.ndarray:
-    sizes = [page_bytes(pool_row_bits[h]) for h in range(len(pool_row_bits))]
+def head_offsets(pool_row_bits, fmt: int = 0) -> np.ndarray:
+    sizes = [page_bytes(pool_row_bits[h], fmt) for h in range(len(pool_row_bits))]
     return np.concatenate([[0], np.cumsum(sizes)[:-1]]).astype(np.int64)
 
 
-def decode_page(page: np.ndarray, row_bits) -> tuple[np.ndarray, np.ndarray]:
+def raw_values(page: np.ndarray, row_bits) -> np.ndarray:
+    """The [128, 128] state of a raw page (binary16 or fp32 rows), as float64."""
+    b = int(np.asarray(row_bits).reshape(-1)[0])
+    dt = np.float16 if b == 16 else np.float32
+    return np.asarray(page, np.uint8)[: D * D * b // 8].view(dt).reshape(D, D).astype(np.float64)
+
+
+def decode_page(page: np.ndarray, row_bits, fmt: int = 0) -> tuple[np.ndarray, np.ndarray]:
     """(scales float32 [128], codes int32 [128, 128]) of one page."""
     page = np.asarray(page, np.uint8)
-    scales = page[: 4 * D].view(np.float32).copy()
+    if fmt == 1:
+        scales = page[: 2 * D].view(np.float16).astype(np.float32)
+    else:
+        scales = page[: 4 * D].view(np.float32).copy()
     codes = np.zeros((D, D), np.int32)
-    offs = row_offsets(row_bits)
+    offs = row_offsets(row_bits, fmt)
     for b in (4, 6, 8):
         rows = np.nonzero(np.asarray(row_bits) == b)[0]
         if len(rows) == 0:
@@ -45,9 +61,9 @@ def decode_page(page: np.ndarray, row_bits) -> tuple[np.ndarray, np.ndarray]:
     return scales, codes
 
 
-def split_slot(slot: np.ndarray, pool_row_bits) -> list[np.ndarray]:
-    offs = head_offsets(pool_row_bits)
-    return [slot[offs[h]: offs[h] + page_bytes(pool_row_bits[h])] for h in range(len(pool_row_bits))]
+def split_slot(slot: np.ndarray, pool_row_bits, fmt: int = 0) -> list[np.ndarray]:
+    offs = head_offsets(pool_row_bits, fmt)
+    return [slot[offs[h]: offs[h] + page_bytes(pool_row_bits[h], fmt)] for h in range(len(pool_row_bits))]
 
 
 class Compare:
@@ -56,14 +72,35 @@ class Compare:
     Tolerances (fp32): y and scales within max relative error 1e-5 per
     (request, head); codes bit-exact except for +-1 at near rounding ties
     (the oracle's quotient within 1e-4 relative of a half-integer), whose
-    count must stay at or below 1e-4 of all codes compared."""
+    count must stay at or below 1e-4 of all codes compared.
 
-    def __init__(self, rtol: float = 1e-5, tie_rel: float = 1e-4, max_tie_frac: float = 1e-4):
+    Binary16 scales must be bit-exact, except a row whose fp32 scale a / q_b
+    lies within 1e-5 relative of a binary16 rounding midpoint: the GPU's a
+    differs from the oracle's by an ulp or two, so it may round to the
+    neighbour; that row's codes are then checked against the GPU's scale.
+
+    Raw pages: fp32 values within 1e-5 of the unit's largest; binary16
+    values bit-exact except where the GPU's value is the binary16 rounding of
+    a value within 4e-6 x max|X| of the unit from X (near a rounding
+    midpoint, or in the subnormal range where the spacing is absolute).  The GPU evaluates X = g x + k u in fp32,
+    whose error is absolute, a few ulps of the largest terms (their
+    magnitude is that of max|X|), and rounds that to binary16, whose spacing
+    at X is 2^-10 |X|: an element flips with probability about
+    2^-10 max|X| / |X|, so the count is bounded by 1e-2 of the values."""
+
+    def __init__(self, rtol: float = 1e-5, tie_rel: float = 1e-4, max_tie_frac: float = 1e-4,
+                 scale_flip_rel: float = 1e-5, raw_tie_rel: float = 4e-6, max_raw_tie_frac: float = 1e-2):
         self.rtol, self.tie_rel, self.max_tie_frac = rtol, tie_rel, max_tie_frac
+        self.scale_flip_rel = scale_flip_rel
+        self.raw_tie_rel, self.max_raw_tie_frac = raw_tie_rel, max_raw_tie_frac
         self.codes = 0
+        self.values = 0
         self.ties = []
+        self.flips = []
+        self.raw_ties = 0
         self.worst_y = 0.0
         self.worst_s = 0.0
+        self.worst_x = 0.0
 
     def y(self, y_gpu, y_ref, where=""):
         y_gpu = np.asarray(y_gpu, np.float64)
@@ -73,33 +110,84 @@ class Compare:
         self.worst_y = max(self.worst_y, err)
         assert err <= self.rtol, f"y rel err {err:.3g} {where}"
 
-    def page(self, page_gpu, page_ref, quot, row_bits, where=""):
-        sg, zg = decode_page(page_gpu, row_bits)
-        sr, zr = decode_page(page_ref, row_bits)
+    def page(self, page_gpu, page_ref, quot, row_bits, where="", fmt=0):
+        sg, zg = decode_page(page_gpu, row_bits, fmt)
+        sr, zr = decode_page(page_ref, row_bits, fmt)
         self.codes += zg.size
-        diff = zg != zr
+        qref = np.asarray(quot, np.float64).copy()
+        zref = zr.copy()
+        if fmt == 1:
+            # binary16 scales: a row whose s = a / q_b lies next to a rounding midpoint of
+            # binary16 may round to the other neighbour on the GPU (its a differs by an ulp
+            # or two); then its codes follow the GPU's scale
+            for i in np.nonzero(sg != sr)[0]:
+                h16 = np.array([sr[i], sg[i]], np.float16).view(np.uint16).astype(np.int64)
+                qb = (1 << (int(row_bits[i]) - 1)) - 1
+                mu = qref[i] * float(sr[i])
+                s = np.abs(mu).max() / qb
+                mid = (float(sr[i]) + float(sg[i])) / 2
+                assert abs(h16[0] - h16[1]) == 1 and abs(s - mid) <= self.scale_flip_rel * s, (
+                    f"scale mismatch row {i} {where}: gpu {sg[i]} ref {sr[i]} (s = {s})")
+                qref[i] = mu / float(sg[i])
+                zref[i] = np.clip(np.rint(qref[i]), -qb, qb)
+                self.flips.append((where, int(i), float(sr[i]), float(sg[i])))
+        diff = zg != zref
         if diff.any():
             ii, jj = np.nonzero(diff)
-            x = quot[ii, jj].astype(np.float64)
+            x = qref[ii, jj]
             frac = np.abs(x - np.floor(x) - 0.5)
             near = frac <= self.tie_rel * np.maximum(np.abs(x), 1.0)
-            one = np.abs(zg[ii, jj] - zr[ii, jj]) == 1
+            one = np.abs(zg[ii, jj] - zref[ii, jj]) == 1
             bad = ~(near & one)
             assert not bad.any(), (
                 f"{int(bad.sum())} code mismatches that are not near-ties {where}: rows {ii[bad][:5]}, "
-                f"cols {jj[bad][:5]}, gpu {zg[ii, jj][bad][:5]}, ref {zr[ii, jj][bad][:5]}, quot {x[bad][:5]}")
+                f"cols {jj[bad][:5]}, gpu {zg[ii, jj][bad][:5]}, ref {zref[ii, jj][bad][:5]}, quot {x[bad][:5]}")
             for a, b in zip(ii, jj):
-                self.ties.append((where, int(a), int(b), float(quot[a, b]), int(zg[a, b]), int(zr[a, b])))
+                self.ties.append((where, int(a), int(b), float(qref[a, b]), int(zg[a, b]), int(zref[a, b])))
+        if fmt == 1:
+            return  # every scale is equal or an accepted flip
         den = np.maximum(np.abs(sr.astype(np.float64)), 1e-38)
         rel = np.abs(sg.astype(np.float64) - sr) / den
         rel[(sr == 0) & (sg == 0)] = 0.0
         self.worst_s = max(self.worst_s, float(rel.max()))
         assert rel.max() <= self.rtol, f"scale rel err {rel.max():.3g} {where}"
 
+    def raw(self, page_gpu, page_ref, quot, row_bits, where=""):
+        """A raw page: fp32 values within rtol of the unit's largest; binary16
+        values equal except where the GPU's value rounds a value within
+        raw_tie_rel x max|X| of X (the oracle's fl32(X), passed as quot)."""
+        xg, xr = raw_values(page_gpu, row_bits), raw_values(page_ref, row_bits)
+        self.values += xg.size
+        if int(np.asarray(row_bits).reshape(-1)[0]) == 32:
+            err = np.abs(xg - xr).max() / max(np.abs(xr).max(), 1e-30)
+            self.worst_x = max(self.worst_x, float(err))
+            assert err <= self.rtol, f"state rel err {err:.3g} {where}"
+            return
+        diff = xg != xr
+        if diff.any():
+            ii, jj = np.nonzero(diff)
+            X = np.asarray(quot, np.float64)
+            x = X[ii, jj]
+            # the GPU's value must be the binary16 rounding of a value within the window of X
+            half_ulp = np.abs(np.spacing(xg[ii, jj].astype(np.float16)).astype(np.float64)) / 2
+            near = np.abs(xg[ii, jj] - x) <= self.raw_tie_rel * np.abs(X).max() + half_ulp
+            bad = ~near
+            assert not bad.any(), (f"{int(bad.sum())} binary16 mismatches beyond the fp32 error window {where}: "
+                                   f"gpu {xg[ii, jj][bad][:5]} ref {xr[ii, jj][bad][:5]} X {x[bad][:5]}")
+            self.raw_ties += len(ii)
+
     def finish(self):
         frac = len(self.ties) / max(self.codes, 1)
         for t in self.ties[:20]:
             print("near-tie:", t)
+        for f in self.flips[:10]:
+            print("binary16 scale flip:", f)
         print(f"codes compared {self.codes}, near-ties {len(self.ties)} ({frac:.2e}), "
-              f"worst y rel {self.worst_y:.2e}, worst scale rel {self.worst_s:.2e}")
+              f"scale flips {len(self.flips)}, raw values {self.values}, raw ties {self.raw_ties}, "
+              f"worst y rel {self.worst_y:.2e}, worst scale rel {self.worst_s:.2e}, "
+              f"worst raw rel {self.worst_x:.2e}")
         assert frac <= self.max_tie_frac, f"tie fraction {frac:.3g} above {self.max_tie_frac}"
+        rows = self.codes // 128
+        assert len(self.flips) <= max(2, 1e-2 * rows), f"{len(self.flips)} scale flips in {rows} rows"
+        rfrac = self.raw_ties / max(self.values, 1)
+        assert rfrac <= self.max_raw_tie_frac, f"raw tie fraction {rfrac:.3g} above {self.max_raw_tie_frac}"

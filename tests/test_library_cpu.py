@@ -72,10 +72,42 @@ def test_desc_validation(bad):
     assert e.value.status == stq.STQ_ERR_ARG
 
 
+def test_desc_bytes_formats():
+    """Binary16 scales save 256 B per page; raw pools are 128 x 128 values of
+    2 or 4 bytes with no scales (the page's fp16 storage and fp32 control)."""
+    bits = np.array([4, 6, 8, 6], np.uint8)
+    _, f32 = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits)
+    _, f16 = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits, flags=stq.STQ_SCALE_F16)
+    assert f32 - f16 == 4 * 256
+    assert f16 == sum(256 + 2048 * int(b) for b in bits)
+    for b in (16, 32):
+        _, slot = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, np.full(4, b, np.uint8))
+        assert slot == 4 * 128 * 128 * b // 8
+        _, slot = stq.stq_desc_bytes(stq.STQ_KDA, 1, 1, 2, np.full(256, b, np.uint8))
+        assert slot == 2 * 128 * 128 * b // 8
+    # the page's compression ratios follow 32 / bits (raw 16: exactly 2x)
+    _, s32 = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, np.full(4, 32, np.uint8))
+    _, s16 = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, np.full(4, 16, np.uint8))
+    assert s32 == 2 * s16
+
+
+@pytest.mark.parametrize("ub, flags, status", [
+    ([16, 16, 8, 16], 0, "STQ_ERR_UNSUPPORTED"),  # raw and quantized units mixed
+    ([32, 16, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),  # two raw widths
+    ([16, 16, 16, 16], 1, "STQ_ERR_ARG"),          # a raw pool has no scales
+    ([6, 6, 6, 6], 2, "STQ_ERR_ARG"),              # unknown flag
+    ([6, 12, 6, 6], 0, "STQ_ERR_ARG"),
+])
+def test_desc_format_validation(ub, flags, status):
+    with pytest.raises(stq.StqError) as e:
+        stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, np.array(ub, np.uint8), flags=flags)
+    assert stq.STATUS[e.value.status] == status
+
+
 def test_unsupported_head_dim():
     L = stq.load()
     ub = np.array([6], np.uint8)
-    d = stq._Desc(0, 1, 1, 1, 64, 64, ub.ctypes.data, None, None)
+    d = stq._Desc(0, 1, 1, 1, 64, 64, ub.ctypes.data, None, None, 0)
     a, b = C.c_size_t(), C.c_size_t()
     assert L.stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)) == stq.STQ_ERR_UNSUPPORTED
 
@@ -117,3 +149,21 @@ def test_page_reader_agrees_with_oracle_packer():
     s, z = decode_page(page, bits)
     np.testing.assert_array_equal(z, want)
     np.testing.assert_array_equal(s, np.arange(128, dtype=np.float32))
+
+
+def test_compare_checks_binary16_pages():
+    """The parity checker accepts identical binary16-scale pages and rejects
+    a planted code change that is not a rounding tie (planted in an
+    oracle-made page, on the CPU)."""
+    import oracle as orc
+    from pages import Compare
+    rng = np.random.default_rng(5)
+    bits = np.full(128, 6, np.uint8)
+    S = rng.standard_normal((128, 128)).astype(np.float32)
+    page, quot, _ = orc.quantize_unit(bits, np.ones(128), np.ones(128), S, with_quot=True, fmt=orc.FMT_F16)
+    cmp = Compare()
+    cmp.page(page, page, quot, bits, fmt=1)
+    bad = page.copy()
+    bad[256] ^= 0x3  # code 0 of row 0 changes by more than one step
+    with pytest.raises(AssertionError):
+        Compare().page(bad, page, quot, bits, fmt=1)
