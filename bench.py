@@ -55,6 +55,7 @@ def parse():
     ap.add_argument("--tokens", type=int, default=256, help="distinct input tokens (cycled)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--no-sweep", action="store_true", help="skip the serving-pool sweep")
+    ap.add_argument("--no-layer-loop", action="store_true", help="skip the 48-layer graph comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     return ap.parse_args()
@@ -390,6 +391,9 @@ def run_ours(args, rank: int, world: int):
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
         sweep = pool_sweep(stq, flush, stream, peak)
+    loop = None
+    if rank == 0 and world == 1 and not args.no_layer_loop:
+        loop = layer_loop(stq, flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -420,6 +424,7 @@ def run_ours(args, rank: int, world: int):
         "gpu_launches": launches,
         "clocks": sampler.summary(),
         "pool_sweep": sweep,
+        "layer_loop": loop,
     }
     print(json.dumps(line), flush=True)
 
@@ -457,6 +462,74 @@ def pool_sweep(stq, flush, stream, peak, reps: int = 20):
         pool.close()
         del x, y
         torch.cuda.empty_cache()
+    return out
+
+
+def layer_loop(stq, flush, layers: int = 48, R: int = 64, reps: int = 20):
+    """Per-layer serving loop: one pool per layer (R requests x 5 slots x 16
+    heads, mixed 6-bit GDN), one token through all layers, each variant
+    captured in one CUDA graph and replayed with the L2 flushed before each
+    replay.  fused: one decode launch per layer.  split: per layer the readout
+    on the main stream and the write-back on a side stream, joined at the end.
+    readout_only: the main-stream half alone (pages unchanged), the path that
+    gates the next layer when the write-backs overlap other work."""
+    import torch
+    wls = [synth.make_workload(4, R=R, H=16, seed=l) for l in range(layers)]
+    pools, idx, xs, ys, us = [], [], [], [], []
+    for w in wls:
+        p = stq.stq_pool_create(w.kind, w.R, w.S, w.H, w.unit_bits, w.row_factor, w.col_factor)
+        pools.append(p)
+        idx.append((torch.arange(w.R, dtype=torch.int32, device="cuda"),
+                    torch.from_numpy(w.slot_of_request.astype(np.int32)).cuda()))
+        inp = w.step_inputs(0)
+        xs.append([torch.from_numpy(inp[k]).cuda() for k in ("q", "k", "v", "beta", "gate")])
+        ys.append(torch.empty((w.R, w.H, 128), dtype=torch.float32, device="cuda"))
+        us.append(torch.empty((w.R, w.H, 128), dtype=torch.float32, device="cuda"))
+    main, side = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def body(kind):
+        for l in range(layers):
+            if kind == "fused":
+                stq.stq_decode_step(pools[l], *idx[l], *xs[l], ys[l], main)
+            elif kind == "split":
+                stq.stq_decode_step_split(pools[l], *idx[l], *xs[l], ys[l], us[l], main, side)
+            else:
+                stq.stq_decode_readout(pools[l], *idx[l], *xs[l], ys[l], us[l], main)
+        if kind == "split":
+            for p in pools:
+                stq.stq_pool_join(p, main)
+
+    out = {"layers": layers, "heads_per_layer": 16, "requests": R, "slots": 5}
+    for kind in ("fused", "split", "readout_only"):
+        torch.cuda.synchronize()
+        with torch.cuda.stream(main):
+            body(kind)  # eager warm-up (sets the kernels' shared-memory attributes)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(main):
+            side.wait_stream(main)
+            g.capture_begin()
+            body(kind)
+            g.capture_end()
+        ts = []
+        for i in range(reps + 3):
+            with torch.cuda.stream(main):
+                flush.zero_()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record(main)
+                g.replay()
+                e.record(main)
+            if i >= 3:
+                ts.append((s, e))
+        torch.cuda.synchronize()
+        med = statistics.median(s.elapsed_time(e) for s, e in ts) * 1e-3
+        out[f"{kind}_graph_us"] = med * 1e6
+        out[f"{kind}_head_steps_per_s"] = layers * R * 16 / med
+        del g
+    for p in pools:
+        stq.stq_pool_check(p)
+        p.close()
+    torch.cuda.empty_cache()
     return out
 
 

@@ -156,6 +156,52 @@ stq_status stq_decode_step(stq_pool *pool, const int32_t *req_idx, const int32_t
                            int32_t n, const float *q, const float *k, const float *v,
                            const float *beta, const float *gate, float *y, void *stream);
 
+/*
+ * The same step split in two ("method steps", steps 3-7, and "technical
+ * novelty" (4): the readout is produced first so that later layers can go
+ * on, while requantisation and write-back run on a separate CUDA stream and
+ * finish before the next step reads the state).  The arithmetic is that of
+ * stq_decode_step, so y, codes and scales are bit-identical to it.
+ *
+ * stq_decode_readout    steps 1-3.  Writes y and u_tilde = u / c, where
+ *                       u = beta (v - k^T D S^), as device fp32 [n][H][128]
+ *                       (16-byte aligned scratch owned by the caller); the
+ *                       pages are only read.
+ * stq_decode_writeback  steps 4-7 with the pool's frozen factors: re-reads
+ *                       the pages of the same entries, forms
+ *                       X = D S^ + k (c u_tilde)^T, requantises and packs it
+ *                       in place.  Reads k, gate and u_tilde (q, v, beta are
+ *                       not read and may be NULL).  The caller orders it after
+ *                       the readout of the same entries and before any other
+ *                       access to their pages.
+ * stq_decode_step_split both halves: the readout on `stream`, the write-back
+ *                       on `side_stream` after an event recorded behind the
+ *                       readout.  The pool then holds a pending write-back:
+ *                       its next asynchronous call makes its own stream wait
+ *                       for it, its synchronous calls (export, import, check)
+ *                       wait for it on the host, and stq_pool_join makes a
+ *                       given stream wait for it.  Before capturing a CUDA
+ *                       graph, join or synchronize any write-back issued
+ *                       outside the capture.
+ * Raw pools (units of 16 or 32 bits) return STQ_ERR_UNSUPPORTED.  Argument
+ * rules are those of stq_decode_step; u_tilde must not be NULL for n > 0.
+ */
+stq_status stq_decode_readout(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                              int32_t n, const float *q, const float *k, const float *v,
+                              const float *beta, const float *gate, float *y, float *u_tilde,
+                              void *stream);
+stq_status stq_decode_writeback(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, const float *k, const float *gate,
+                                const float *u_tilde, void *stream);
+stq_status stq_decode_step_split(stq_pool *pool, const int32_t *req_idx,
+                                 const int32_t *slot_idx, int32_t n, const float *q,
+                                 const float *k, const float *v, const float *beta,
+                                 const float *gate, float *y, float *u_tilde, void *stream,
+                                 void *side_stream);
+
+/* Make `stream` wait for the pool's pending split write-back (no-op if none). */
+stq_status stq_pool_join(stq_pool *pool, void *stream);
+
 /* Copy one slot's raw pages (per_slot_bytes bytes) to / from host memory.
  * Synchronous (device-wide ordering with the legacy default stream). */
 stq_status stq_export_slot(const stq_pool *pool, int32_t req, int32_t slot, void *host_dst,
@@ -163,7 +209,7 @@ stq_status stq_export_slot(const stq_pool *pool, int32_t req, int32_t slot, void
 stq_status stq_import_slot(stq_pool *pool, int32_t req, int32_t slot, const void *host_src,
                            size_t bytes);
 
-/* Synchronize `stream`, then return and clear the pool's device error word
+/* Synchronize `stream` (and any pending split write-back), then return and clear the pool's device error word
  * (STQ_ERR_INDEX, STQ_ERR_NONFINITE or STQ_ERR_TIMEOUT; STQ_OK if clear). */
 stq_status stq_pool_check(stq_pool *pool, void *stream);
 

@@ -20,6 +20,9 @@ struct stq_pool {
     uint8_t *d_pages = nullptr;
     void *d_tables = nullptr;
     uint32_t *d_err = nullptr;
+    // split decode: events behind the last readout and the last write-back
+    cudaEvent_t ev_read = nullptr, ev_wb = nullptr;
+    mutable bool wb_pending = false;
     stq::Tables t{};
     std::vector<uint32_t> head_off, page_bytes;
 };
@@ -187,6 +190,47 @@ stq_status check_launch_args(const stq_pool *p, const int32_t *req, const int32_
     return STQ_OK;
 }
 
+// A pending split write-back is ordered before the next access: asynchronous
+// calls make their stream wait for it, synchronous ones wait on the host.
+cudaError_t join_async(const stq_pool *p, cudaStream_t stream)
+{
+    if (!p->wb_pending) return cudaSuccess;
+    cudaError_t e = cudaStreamWaitEvent(stream, p->ev_wb, 0);
+    if (e == cudaSuccess) p->wb_pending = false;
+    return e;
+}
+
+cudaError_t join_host(const stq_pool *p)
+{
+    if (!p->wb_pending) return cudaSuccess;
+    cudaError_t e = cudaEventSynchronize(p->ev_wb);
+    if (e == cudaSuccess) p->wb_pending = false;
+    return e;
+}
+
+stq_status check_decode_args(const stq_pool *p, const int32_t *req, const int32_t *slot, int32_t n,
+                             const float *q, const float *k, const float *v, const float *beta,
+                             const float *gate, const float *y)
+{
+    stq_status st = check_launch_args(p, req, slot, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && (!q || !k || !v || !beta || !gate || !y))
+        return fail(STQ_ERR_ARG, "a q/k/v/beta/gate/y pointer is NULL");
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
+                          reinterpret_cast<uintptr_t>(v) |
+                          (p->kind == STQ_KDA ? reinterpret_cast<uintptr_t>(gate) : 0);
+    if (mis % 16 != 0) return fail(STQ_ERR_ARG, "q, k, v (and the KDA gate) must be 16-byte aligned");
+    return STQ_OK;
+}
+
+stq_status check_split_args(const stq_pool *p, int32_t n, const float *u_tilde)
+{
+    if (p->raw_bits) return fail(STQ_ERR_UNSUPPORTED, "split decode needs a quantized pool");
+    if (n > 0 && u_tilde == nullptr) return fail(STQ_ERR_ARG, "u_tilde is NULL");
+    if (reinterpret_cast<uintptr_t>(u_tilde) % 16 != 0) return fail(STQ_ERR_ARG, "u_tilde not 16-byte aligned");
+    return STQ_OK;
+}
+
 }  // namespace
 
 namespace stq {
@@ -324,6 +368,9 @@ stq_status stq_pool_destroy(stq_pool *p)
 {
     if (p == nullptr) return STQ_OK;
     DeviceGuard g(p->device);
+    if (p->wb_pending) cudaEventSynchronize(p->ev_wb);
+    if (p->ev_read) cudaEventDestroy(p->ev_read);
+    if (p->ev_wb) cudaEventDestroy(p->ev_wb);
     cudaFree(p->d_pages);
     cudaFree(p->d_tables);
     cudaFree(p->d_err);
@@ -360,7 +407,9 @@ stq_status stq_quantize_state(stq_pool *p, const int32_t *req_idx, const int32_t
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
-    cudaError_t e = stq::launch_quantize(view(p), req_idx, slot_idx, n, state, (cudaStream_t)stream);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = stq::launch_quantize(view(p), req_idx, slot_idx, n, state, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "quantize launch");
 }
 
@@ -376,8 +425,9 @@ stq_status stq_dequantize_state(stq_pool *p, const int32_t *req_idx, const int32
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
-    cudaError_t e =
-        stq::launch_dequantize(view(p), req_idx, slot_idx, n, state_out, (cudaStream_t)stream);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = stq::launch_dequantize(view(p), req_idx, slot_idx, n, state_out, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "dequantize launch");
 }
 
@@ -385,24 +435,105 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
                            int32_t n, const float *q, const float *k, const float *v,
                            const float *beta, const float *gate, float *y, void *stream)
 {
-    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    stq_status st = check_decode_args(p, req_idx, slot_idx, n, q, k, v, beta, gate, y);
     if (st != STQ_OK) return st;
-    if (n > 0 && (!q || !k || !v || !beta || !gate || !y))
-        return fail(STQ_ERR_ARG, "a q/k/v/beta/gate/y pointer is NULL");
-    {
-        const uintptr_t mis = reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k) |
-                              reinterpret_cast<uintptr_t>(v) |
-                              (p != nullptr && p->kind == STQ_KDA ? reinterpret_cast<uintptr_t>(gate) : 0);
-        if (mis % 16 != 0) return fail(STQ_ERR_ARG, "q, k, v (and the KDA gate) must be 16-byte aligned");
-    }
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
-    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y};
-    cudaError_t e = p->raw_bits ? stq::launch_decode_raw(view(p), io, (cudaStream_t)stream)
-                                : stq::launch_decode(view(p), io, (cudaStream_t)stream);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, nullptr};
+    e = p->raw_bits ? stq::launch_decode_raw(view(p), io, (cudaStream_t)stream)
+                    : stq::launch_decode(view(p), io, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "decode launch");
+}
+
+stq_status stq_decode_readout(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                              int32_t n, const float *q, const float *k, const float *v,
+                              const float *beta, const float *gate, float *y, float *u_tilde,
+                              void *stream)
+{
+    stq_status st = check_decode_args(p, req_idx, slot_idx, n, q, k, v, beta, gate, y);
+    if (st != STQ_OK) return st;
+    st = check_split_args(p, n, u_tilde);
+    if (st != STQ_OK) return st;
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u_tilde};
+    e = stq::launch_decode_readout(view(p), io, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "readout launch");
+}
+
+stq_status stq_decode_writeback(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, const float *k, const float *gate,
+                                const float *u_tilde, void *stream)
+{
+    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && (!k || !gate)) return fail(STQ_ERR_ARG, "k or gate is NULL");
+    const uintptr_t mis = reinterpret_cast<uintptr_t>(k) |
+                          (p->kind == STQ_KDA ? reinterpret_cast<uintptr_t>(gate) : 0);
+    if (mis % 16 != 0) return fail(STQ_ERR_ARG, "k (and the KDA gate) must be 16-byte aligned");
+    st = check_split_args(p, n, u_tilde);
+    if (st != STQ_OK) return st;
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    // the write-back reads u~ through the v slot; q and beta are not read
+    stq::DecodeIO io{req_idx, slot_idx, n, nullptr, k, u_tilde, nullptr, gate, nullptr, nullptr};
+    e = stq::launch_decode_writeback(view(p), io, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "write-back launch");
+}
+
+stq_status stq_decode_step_split(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                                 int32_t n, const float *q, const float *k, const float *v,
+                                 const float *beta, const float *gate, float *y, float *u_tilde,
+                                 void *stream, void *side_stream)
+{
+    stq_status st = check_decode_args(p, req_idx, slot_idx, n, q, k, v, beta, gate, y);
+    if (st != STQ_OK) return st;
+    st = check_split_args(p, n, u_tilde);
+    if (st != STQ_OK) return st;
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    cudaError_t e = cudaSuccess;
+    if (p->ev_read == nullptr) e = cudaEventCreateWithFlags(&p->ev_read, cudaEventDisableTiming);
+    if (e == cudaSuccess && p->ev_wb == nullptr) e = cudaEventCreateWithFlags(&p->ev_wb, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "event create");
+    const cudaStream_t s0 = (cudaStream_t)stream, s1 = (cudaStream_t)side_stream;
+    e = join_async(p, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u_tilde};
+    e = stq::launch_decode_readout(view(p), io, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "readout launch");
+    e = cudaEventRecord(p->ev_read, s0);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s1, p->ev_read, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "readout event");
+    stq::DecodeIO wb{req_idx, slot_idx, n, nullptr, k, u_tilde, nullptr, gate, nullptr, nullptr};
+    e = stq::launch_decode_writeback(view(p), wb, s1);
+    if (e != cudaSuccess) return cuda_fail(e, "write-back launch");
+    e = cudaEventRecord(p->ev_wb, s1);
+    if (e != cudaSuccess) return cuda_fail(e, "write-back event");
+    p->wb_pending = true;
+    return STQ_OK;
+}
+
+stq_status stq_pool_join(stq_pool *p, void *stream)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    DeviceGuard g(p->device);
+    cudaError_t e = join_async(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "wait for the pending write-back");
 }
 
 stq_status stq_export_slot(const stq_pool *p, int32_t req, int32_t slot, void *host_dst,
@@ -415,7 +546,8 @@ stq_status stq_export_slot(const stq_pool *p, int32_t req, int32_t slot, void *h
         return fail(STQ_ERR_ARG, "bytes = %zu, slot holds %zu", bytes, p->slot_bytes);
     DeviceGuard g(p->device);
     const uint8_t *src = p->d_pages + ((size_t)req * p->S + slot) * p->slot_bytes;
-    cudaError_t e = cudaMemcpy(host_dst, src, bytes, cudaMemcpyDeviceToHost);
+    cudaError_t e = join_host(p);
+    if (e == cudaSuccess) e = cudaMemcpy(host_dst, src, bytes, cudaMemcpyDeviceToHost);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "export");
 }
 
@@ -429,7 +561,8 @@ stq_status stq_import_slot(stq_pool *p, int32_t req, int32_t slot, const void *h
         return fail(STQ_ERR_ARG, "bytes = %zu, slot holds %zu", bytes, p->slot_bytes);
     DeviceGuard g(p->device);
     uint8_t *dst = p->d_pages + ((size_t)req * p->S + slot) * p->slot_bytes;
-    cudaError_t e = cudaMemcpy(dst, host_src, bytes, cudaMemcpyHostToDevice);
+    cudaError_t e = join_host(p);
+    if (e == cudaSuccess) e = cudaMemcpy(dst, host_src, bytes, cudaMemcpyHostToDevice);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "import");
 }
 
@@ -438,6 +571,7 @@ stq_status stq_pool_check(stq_pool *p, void *stream)
     if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
     DeviceGuard g(p->device);
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e == cudaSuccess) e = join_host(p);
     if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
     uint32_t word = 0;
     e = cudaMemcpy(&word, p->d_err, 4, cudaMemcpyDeviceToHost);

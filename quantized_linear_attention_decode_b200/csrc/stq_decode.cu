@@ -23,6 +23,14 @@
 // mantissa of 2^23, then 2^23 + 2^(b-1) subtracted), pairs of columns are
 // processed with packed fma.rn.f32x2, and requantised codes are read back
 // from the mantissa of fma(w, inv, 2^23 + 2^(b-1)).
+//
+// The same kernel, instantiated per mode, also runs the step split in two
+// ("method steps", steps 3-7: the readout first, the requantisation and
+// write-back on a separate stream): kReadout stops after the column epilogue
+// and stores u~ = u / c per tile; kWriteback re-reads the page, takes u~ from
+// that buffer in place of the column sums, and runs pass 2.  Both halves do
+// the fused kernel's arithmetic, so the split step's y, codes and scales are
+// bit-identical to the fused step's.
 #include <cstddef>
 #include <cstdint>
 
@@ -34,6 +42,11 @@ namespace stq {
 namespace {
 
 constexpr int kThreads = 256;
+
+// kernel modes
+constexpr int kFused = 0;      // the whole step (one state traversal)
+constexpr int kReadout = 1;    // steps 1-3: y and u~; the page is only read
+constexpr int kWriteback = 2;  // steps 4-7 given u~: requantise and pack in place
 constexpr int kStages = 4;
 constexpr int kMaxPage = kScaleBytes + 16 * 8 * kD;    // 16896: every row at 8 bits
 constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
@@ -370,7 +383,7 @@ __device__ __forceinline__ float magic_out(int b)
 // Pass 1: unpack the old codes, accumulate the two column sums and leave
 // per-warp partials in red.  B = 4, 6, 8: every row has B
 // bits (GDN); B = 0: per-row widths (KDA).
-template <int B, int SB>
+template <int B, int SB, bool ACC = true>
 __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -385,33 +398,43 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
         const int i = i0 + ii;
         if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + 16 * B * i, cg, z[ii]);
         else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
-        const float4 kl = R.kl[i];
+        if constexpr (ACC) {
+            const float4 kl = R.kl[i];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            av[p] = ffma2(make_float2(kl.x, kl.y), z[ii][p], av[p]);
-            ay[p] = ffma2(make_float2(kl.z, kl.w), z[ii][p], ay[p]);
+            for (int p = 0; p < 4; ++p) {
+                av[p] = ffma2(make_float2(kl.x, kl.y), z[ii][p], av[p]);
+                ay[p] = ffma2(make_float2(kl.z, kl.w), z[ii][p], ay[p]);
+            }
         }
     }
+    if constexpr (ACC) {
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        av[p] = fadd2(av[p], make_float2(__shfl_xor_sync(0xffffffffu, av[p].x, 16),
-                                         __shfl_xor_sync(0xffffffffu, av[p].y, 16)));
-        ay[p] = fadd2(ay[p], make_float2(__shfl_xor_sync(0xffffffffu, ay[p].x, 16),
-                                         __shfl_xor_sync(0xffffffffu, ay[p].y, 16)));
+        for (int p = 0; p < 4; ++p) {
+            av[p] = fadd2(av[p], make_float2(__shfl_xor_sync(0xffffffffu, av[p].x, 16),
+                                             __shfl_xor_sync(0xffffffffu, av[p].y, 16)));
+            ay[p] = fadd2(ay[p], make_float2(__shfl_xor_sync(0xffffffffu, ay[p].x, 16),
+                                             __shfl_xor_sync(0xffffffffu, ay[p].y, 16)));
+        }
+        // half 0 keeps the v-sums, half 1 the y-sums; column j of a sum sits at
+        // ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3) (conflict-free 16-byte stores)
+        const float2 *src = rgl == 0 ? av : ay;
+        float *dst = &sm.red[warp * 256 + rgl * 128 + cg * 4];
+        *reinterpret_cast<float4 *>(dst) = make_float4(src[0].x, src[0].y, src[1].x, src[1].y);
+        *reinterpret_cast<float4 *>(dst + 64) = make_float4(src[2].x, src[2].y, src[3].x, src[3].y);
     }
-    // half 0 keeps the v-sums, half 1 the y-sums; column j of a sum sits at
-    // ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3) (conflict-free 16-byte stores)
-    const float2 *src = rgl == 0 ? av : ay;
-    float *dst = &sm.red[warp * 256 + rgl * 128 + cg * 4];
-    *reinterpret_cast<float4 *>(dst) = make_float4(src[0].x, src[0].y, src[1].x, src[1].y);
-    *reinterpret_cast<float4 *>(dst + 64) = make_float4(src[2].x, src[2].y, src[3].x, src[3].y);
 }
 
-// Per column (threads 0..127): v_old, u, y, u / c.
+// Per column (threads 0..127): v_old, u, y, u / c.  The write-back takes
+// u / c from the readout's buffer (prefetched into the stage's v) instead.
+template <int MODE>
 __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const RowCoef &R,
                                                 const DecodeIO &io, int tile, float beta)
 {
     const int j = threadIdx.x;
+    if (MODE == kWriteback) {
+        sm.ut[j] = S.v[j];
+        return;
+    }
     const int at = ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3);
     float vz = 0.0f, yz = 0.0f;
 #pragma unroll
@@ -424,13 +447,15 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     const float kq = (R.kqp[0] + R.kqp[1]) + (R.kqp[2] + R.kqp[3]);
     const float yj = fmaf(u, kq, cj * yz);
     io.y[static_cast<size_t>(tile) * kD + j] = yj;
-    sm.ut[j] = u * rcp_approx(cj);
+    const float ut = u * rcp_approx(cj);
+    if (MODE == kReadout) io.u_out[static_cast<size_t>(tile) * kD + j] = ut;
+    else sm.ut[j] = ut;
     if (!isfinite(u) || !isfinite(yj)) atomicOr(&sm.flags, kErrNonFinite);
 }
 
 // Per row (threads 128..255) of the next tile: decayed scale e_i and the
 // coefficients both passes need; warp 4 also forms k.q.
-template <int KIND, int SB>
+template <int KIND, int SB, int MODE>
 __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, int s)
 {
     const int r = threadIdx.x - kD;
@@ -446,7 +471,8 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     const float rr = S.r[r];
     const float e = (g * sc) * rr;
     const float kr = S.k[r];
-    const float ka = kr * e, la = S.q[r] * e;
+    const float qr = MODE == kWriteback ? 0.0f : S.q[r];  // the write-back loads no q
+    const float ka = kr * e, la = qr * e;
     const float hq = kr * rcp_approx(e);
     const bool dropped = !(e != 0.0f && fabsf(hq) <= 1e30f);
     R.kl[r] = make_float4(ka, ka, la, la);
@@ -457,7 +483,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     const uint32_t bal = __ballot_sync(0xffffffffu, dropped);
     if ((r & 31) == 0) R.deg[r >> 5] = bal;
     if (!isfinite(e)) atomicOr(&sm.flags, kErrNonFinite);
-    float a = kr * S.q[r];
+    float a = kr * qr;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
     if ((r & 31) == 0) R.kqp[r >> 5] = a;
@@ -661,7 +687,7 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
 // i + 3 into its stage, and the raw location {req, slot, head offset, page
 // bytes} of tile i + 5 = (request entry n5, head h5).  The small copies are
 // spread over warps 5-7, which have the least other work at this point.
-template <int KIND>
+template <int KIND, int MODE>
 __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const DecodeIO &io, int i, int t3, int t5,
                                          int n5, int h5, int tiles)
 {
@@ -669,13 +695,15 @@ __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const Deco
     if (t3 < tiles) {
         Stage &S = sm.st[(i + 3) % kStages];
         const size_t base = static_cast<size_t>(t3) * kD + 4 * (t & 31);
-        if (t < 32) cp_async16(&S.q[4 * t], io.q + base);
+        if (t < 32) {
+            if (MODE != kWriteback) cp_async16(&S.q[4 * t], io.q + base);
+        }
         else if (t < 64) cp_async16(&S.k[4 * (t - 32)], io.k + base);
         else if (t < 96) cp_async16(&S.v[4 * (t - 64)], io.v + base);
         else if (t < 128) {
             if (KIND == STQ_KDA) cp_async16(&S.g[4 * (t - 96)], io.gate + base);
         } else if (t == 160) {
-            cp_async4(&sm.beta[(i + 3) % kStages], io.beta + t3);
+            if (MODE != kWriteback) cp_async4(&sm.beta[(i + 3) % kStages], io.beta + t3);
         } else if (t == 192) {
             if (KIND == STQ_GDN) cp_async4(&sm.alpha[(i + 3) % kStages], io.gate + t3);
         }
@@ -693,21 +721,21 @@ __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const Deco
 }
 
 // Synchronous fill of a stage's vectors and beta/alpha (first tiles only).
-template <int KIND>
+template <int KIND, int MODE>
 __device__ __forceinline__ void fill_sync(Smem &sm, const DecodeIO &io, int s, int tile)
 {
     const int t = threadIdx.x;
     Stage &S = sm.st[s];
     const size_t base = static_cast<size_t>(tile) * kD;
     if (t < kD) {
-        S.q[t] = io.q[base + t];
+        if (MODE != kWriteback) S.q[t] = io.q[base + t];
         S.k[t] = io.k[base + t];
     } else {
         S.v[t - kD] = io.v[base + t - kD];
         if (KIND == STQ_KDA) S.g[t - kD] = io.gate[base + t - kD];
     }
     if (t == 0) {
-        sm.beta[s] = io.beta[tile];
+        sm.beta[s] = MODE != kWriteback ? io.beta[tile] : 0.0f;
         sm.alpha[s] = KIND == STQ_GDN ? io.gate[tile] : 0.0f;
     }
 }
@@ -734,7 +762,7 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
 // A stage is last read before the second barrier of its tile (pass 2 reads
 // only registers and the row data); thread 96 refills it after the first
 // barrier of the next tile.
-template <int KIND, int SB>
+template <int KIND, int SB, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -766,12 +794,12 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
     }
     for (int a = 0; a < 3; ++a)
-        if (first + a * G < tiles) fill_sync<KIND>(sm, io, a, first + a * G);
+        if (first + a * G < tiles) fill_sync<KIND, MODE>(sm, io, a, first + a * G);
     __syncthreads();
     bool timed_out = false;
     if (tid >= kD) {
         // warp-uniform outcome: row_setup's shuffles need every lane
-        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB>(sm, sm.st[0], sm.rc[0], 0);
+        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB, MODE>(sm, sm.st[0], sm.rc[0], 0);
         else timed_out = true;
     }
     timed_out = __syncthreads_or(timed_out) != 0;
@@ -788,17 +816,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         const bool valid = R.valid != 0;
         const int b = valid ? R.bits[0] : 8;
         float2 z[8][4];
+        constexpr bool kAcc = MODE != kWriteback;
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0, SB>(sm, S, R, z);
-            else if (b == 8) pass1<8, SB>(sm, S, R, z);
-            else if (b == 6) pass1<6, SB>(sm, S, R, z);
-            else pass1<4, SB>(sm, S, R, z);
+            if (KIND == STQ_KDA) pass1<0, SB, kAcc>(sm, S, R, z);
+            else if (b == 8) pass1<8, SB, kAcc>(sm, S, R, z);
+            else if (b == 6) pass1<6, SB, kAcc>(sm, S, R, z);
+            else pass1<4, SB, kAcc>(sm, S, R, z);
         }
         cp_async_wait<1>();
         __syncthreads();
         if (tid == 96 && tile + 3 * G < tiles)  // warp 3: no vector prefetch for GDN
             issue<KIND>(sm, (i + 3) % kStages, p, resolve(p, raw_from_smem(sm, i + 3)));
-        prefetch<KIND>(sm, p, io, i, tile + 3 * G, tile + 5 * G, n5, h5, tiles);
+        prefetch<KIND, MODE>(sm, p, io, i, tile + 3 * G, tile + 5 * G, n5, h5, tiles);
         n5 += gq;
         h5 += gr;
         if (h5 >= p.H) {
@@ -807,16 +836,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         bool tout = false;
         if (tid < kD) {
-            if (valid) column_epilogue(sm, S, R, io, tile, sm.beta[s]);
+            if (valid) column_epilogue<MODE>(sm, S, R, io, tile, sm.beta[s]);
         } else if (tile + G < tiles) {
             const int sn = (i + 1) % kStages;
             if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)))
-                row_setup<KIND, SB>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
+                row_setup<KIND, SB, MODE>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
             else
                 tout = true;
         }
         timed_out = __syncthreads_or(tout) != 0;
-        if (valid) {
+        if (valid && MODE != kReadout) {
             if (KIND == STQ_KDA) pass2<0, SB>(sm, R, z);
             else if (b == 8) pass2<8, SB>(sm, R, z);
             else if (b == 6) pass2<6, SB>(sm, R, z);
@@ -842,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
 
 constexpr int kMaxDevices = 64;
 
-template <int KIND, int SB>
+template <int KIND, int SB, int MODE>
 cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
     // per device: SM count, and the dynamic shared-memory opt-in of this kernel
@@ -856,24 +885,40 @@ cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(decode_kernel<KIND, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<KIND, SB, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         sms[dev] = n > 0 ? n : 148;
     }
     const int tiles = io.n * p.H;
     const int grid = tiles < 2 * sms[dev] ? tiles : 2 * sms[dev];
-    decode_kernel<KIND, SB><<<grid, kThreads, smem, stream>>>(p, io, tiles);
+    decode_kernel<KIND, SB, MODE><<<grid, kThreads, smem, stream>>>(p, io, tiles);
     count_launch();
     return cudaGetLastError();
+}
+
+template <int MODE>
+cudaError_t launch_mode(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
+{
+    if (p.scale_bytes == 2)
+        return p.kind == STQ_KDA ? launch<STQ_KDA, 2, MODE>(p, io, stream) : launch<STQ_GDN, 2, MODE>(p, io, stream);
+    return p.kind == STQ_KDA ? launch<STQ_KDA, 4, MODE>(p, io, stream) : launch<STQ_GDN, 4, MODE>(p, io, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
-    if (p.scale_bytes == 2)
-        return p.kind == STQ_KDA ? launch<STQ_KDA, 2>(p, io, stream) : launch<STQ_GDN, 2>(p, io, stream);
-    return p.kind == STQ_KDA ? launch<STQ_KDA, 4>(p, io, stream) : launch<STQ_GDN, 4>(p, io, stream);
+    return launch_mode<kFused>(p, io, stream);
+}
+
+cudaError_t launch_decode_readout(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
+{
+    return launch_mode<kReadout>(p, io, stream);
+}
+
+cudaError_t launch_decode_writeback(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
+{
+    return launch_mode<kWriteback>(p, io, stream);
 }
 
 }  // namespace stq

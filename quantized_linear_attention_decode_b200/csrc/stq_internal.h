@@ -53,12 +53,15 @@ struct DecodeIO {
     const int32_t *req_idx;
     const int32_t *slot_idx;
     int n;
-    const float *q, *k, *v, *beta, *gate;
+    const float *q, *k, *v, *beta, *gate;  // the write-back reads u~ through v (q, beta unused)
     float *y;
+    float *u_out;  // the readout's u~ = u / c per tile [n][H][128]; unused by the other modes
 };
 
 cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+cudaError_t launch_decode_readout(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+cudaError_t launch_decode_writeback(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                             int n, const float *state, cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,

@@ -24,6 +24,7 @@ STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE
 # every symbol include/stq.h declares
 EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
            "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
+           "stq_decode_readout", "stq_decode_writeback", "stq_decode_step_split", "stq_pool_join",
            "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
            "stq_status_str", "stq_last_error")
 
@@ -63,6 +64,10 @@ def load():
         "stq_quantize_state": [P, P, P, I32, P, P],
         "stq_dequantize_state": [P, P, P, I32, P, P],
         "stq_decode_step": [P, P, P, I32, P, P, P, P, P, P, P],
+        "stq_decode_readout": [P, P, P, I32, P, P, P, P, P, P, P, P],
+        "stq_decode_writeback": [P, P, P, I32, P, P, P, P],
+        "stq_decode_step_split": [P, P, P, I32, P, P, P, P, P, P, P, P, P],
+        "stq_pool_join": [P, P],
         "stq_export_slot": [P, I32, I32, P, SZ],
         "stq_import_slot": [P, I32, I32, P, SZ],
         "stq_pool_check": [P, P],
@@ -215,6 +220,48 @@ def stq_decode_step(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, strea
         pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
         _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
         _stream(stream)))
+
+
+def _vecs(pool, n):
+    vec = (n, pool.H, 128)
+    return vec, ((n, pool.H) if pool.kind == STQ_GDN else vec)
+
+
+def stq_decode_readout(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, u_tilde, stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    f = torch.float32
+    vec, gshape = _vecs(pool, n)
+    _check(load().stq_decode_readout(
+        pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
+        _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
+        _dev(u_tilde, f, vec, "u_tilde"), _stream(stream)))
+
+
+def stq_decode_writeback(pool: Pool, req_idx, slot_idx, k, gate, u_tilde, stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    f = torch.float32
+    vec, gshape = _vecs(pool, n)
+    _check(load().stq_decode_writeback(
+        pool.handle, r, s, n, _dev(k, f, vec, "k"), _dev(gate, f, gshape, "gate"),
+        _dev(u_tilde, f, vec, "u_tilde"), _stream(stream)))
+
+
+def stq_decode_step_split(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, u_tilde, stream=None,
+                          side_stream=None) -> None:
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    f = torch.float32
+    vec, gshape = _vecs(pool, n)
+    _check(load().stq_decode_step_split(
+        pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
+        _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
+        _dev(u_tilde, f, vec, "u_tilde"), _stream(stream), _stream(side_stream)))
+
+
+def stq_pool_join(pool: Pool, stream=None) -> None:
+    _check(load().stq_pool_join(pool.handle, _stream(stream)))
 
 
 def stq_export_slot(pool: Pool, req: int, slot: int) -> np.ndarray:

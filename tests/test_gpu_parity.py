@@ -38,12 +38,28 @@ def _init(wl, pool):
     return req, slot
 
 
-def _step(wl, pool, req, slot, t, requests=None):
+_side = None
+
+
+def side_stream():
+    global _side
+    if _side is None:
+        _side = torch.cuda.Stream()
+    return _side
+
+
+def _step(wl, pool, req, slot, t, requests=None, split=False):
+    """One decode token: the fused step, or (split=True) the readout on the
+    current stream and the write-back on a side stream."""
     inp = wl.step_inputs(t, requests)
     n = len(inp["beta"])
     y = torch.empty((n, wl.H, 128), dtype=torch.float32, device="cuda")
-    stq.stq_decode_step(pool, req, slot, _cuda(inp["q"]), _cuda(inp["k"]), _cuda(inp["v"]),
-                        _cuda(inp["beta"]), _cuda(inp["gate"]), y)
+    x = [_cuda(inp[key]) for key in ("q", "k", "v", "beta", "gate")]
+    if split:
+        u = torch.empty((n, wl.H, 128), dtype=torch.float32, device="cuda")
+        stq.stq_decode_step_split(pool, req, slot, *x, y, u, side_stream=side_stream())
+    else:
+        stq.stq_decode_step(pool, req, slot, *x, y)
     stq.stq_pool_check(pool)
     return inp, y.cpu().numpy()
 
@@ -55,7 +71,7 @@ def _oracle_unit(wl, rb, page, inp, a, h):
                          page, inp["q"][a, h], inp["k"][a, h], inp["v"][a, h], inp["beta"][a, h], g)
 
 
-def _teacher_forced(wl, steps, units=None, check_steps=None):
+def _teacher_forced(wl, steps, units=None, check_steps=None, split=False):
     """Runs `steps` decode steps on all requests; checks `units` ((request,
     head) pairs, default all) at `check_steps` (default all)."""
     pool = _pool(wl)
@@ -68,7 +84,7 @@ def _teacher_forced(wl, steps, units=None, check_steps=None):
         check = check_steps is None or t in check_steps
         before = {a: split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb)
                   for a in reqs_checked} if check else None
-        inp, y = _step(wl, pool, req, slot, t)
+        inp, y = _step(wl, pool, req, slot, t, split=split)
         if not check:
             continue
         for a in reqs_checked:
