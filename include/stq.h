@@ -199,6 +199,30 @@ stq_status stq_decode_step_split(stq_pool *pool, const int32_t *req_idx,
                                  const float *gate, float *y, float *u_tilde, void *stream,
                                  void *side_stream);
 
+/*
+ * The split step with scratch the library owns: no counterpart in the paper.
+ * For callers that must not allocate device memory while they run, such as a
+ * serving engine that reserved all of its device memory at start-up, or one
+ * that cannot risk an allocation failing under memory pressure or stalling
+ * the device inside its latency budget.  Same arguments and results as
+ * stq_decode_step; it runs stq_decode_readout and stq_decode_writeback one
+ * after the other on `stream`, with u_tilde kept in a fixed 4 MiB device array
+ * built into the library (every GPU that loads the library holds it until the
+ * process exits).  It never allocates or frees memory.
+ *   - n * H may be at most 8192 tiles (n * H * 128 floats <= 2^20);
+ *     larger calls return STQ_ERR_ARG before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device); make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls that may overlap on the
+ *     GPU (other streams, other threads) race on it and must be serialized by
+ *     the caller.  Each call writes the array in full before reading it, so
+ *     nothing has to be cleared between calls.
+ * Raw pools return STQ_ERR_UNSUPPORTED.
+ */
+stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                                  int32_t n, const float *q, const float *k, const float *v,
+                                  const float *beta, const float *gate, float *y, void *stream);
+
 /* Make `stream` wait for the pool's pending split write-back (no-op if none). */
 stq_status stq_pool_join(stq_pool *pool, void *stream);
 

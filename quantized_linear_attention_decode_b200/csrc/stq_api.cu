@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -526,6 +527,77 @@ stq_status stq_decode_step_split(stq_pool *p, const int32_t *req_idx, const int3
     if (e != cudaSuccess) return cuda_fail(e, "write-back event");
     p->wb_pending = true;
     return STQ_OK;
+}
+
+// ---------------------------------------------------------------- decode with built-in scratch
+//
+// The split step needs a per-tile u~ buffer between its two kernels.  Callers
+// that cannot allocate device memory while they run (an engine that has
+// reserved all of its device memory up front, or one whose latency budget
+// cannot absorb an allocation, which may fail under memory pressure or wait
+// for the whole device) can use stq_decode_step_static instead: it runs both
+// kernels on one stream and keeps u~ in the fixed array below.  The array is
+// part of the library's device image, so every GPU that loads the library
+// holds its 4 MiB until the process exits.
+
+}  // extern "C"
+
+static __device__ __align__(256) float g_static_u_tilde[stq::kStaticScratchFloats];
+
+namespace {
+
+constexpr int kMaxScratchDevices = 64;
+float *g_static_u_tilde_ptr[kMaxScratchDevices] = {};
+std::mutex g_static_mu;
+
+// Device address of the array on the current device, looked up once per
+// device.  In host code the array's name only stands for the symbol.
+cudaError_t static_u_tilde(int dev, float **out)
+{
+    if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_u_tilde_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_u_tilde);
+        if (e != cudaSuccess) return e;
+        g_static_u_tilde_ptr[dev] = static_cast<float *>(ptr);
+    }
+    *out = g_static_u_tilde_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" {
+
+stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                                  int32_t n, const float *q, const float *k, const float *v,
+                                  const float *beta, const float *gate, float *y, void *stream)
+{
+    stq_status st = check_decode_args(p, req_idx, slot_idx, n, q, k, v, beta, gate, y);
+    if (st != STQ_OK) return st;
+    if (p->raw_bits) return fail(STQ_ERR_UNSUPPORTED, "the built-in scratch decode needs a quantized pool");
+    const long long need = (long long)n * p->H * kD;
+    if (need > (long long)stq::kStaticScratchFloats)
+        return fail(STQ_ERR_ARG, "n * H = %lld tiles exceeds the built-in scratch of %lld tiles",
+                    (long long)n * p->H, (long long)(stq::kStaticScratchFloats / kD));
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    float *u = nullptr;
+    cudaError_t e = static_u_tilde(p->device, &u);
+    if (e != cudaSuccess) return cuda_fail(e, "address of the built-in scratch");
+    const cudaStream_t s0 = (cudaStream_t)stream;
+    e = join_async(p, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    // the readout fills u~ for every tile of the call before the write-back reads it
+    stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u};
+    e = stq::launch_decode_readout(view(p), io, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "readout launch");
+    stq::DecodeIO wb{req_idx, slot_idx, n, nullptr, k, u, nullptr, gate, nullptr, nullptr};
+    e = stq::launch_decode_writeback(view(p), wb, s0);
+    return e == cudaSuccess ? STQ_OK : cuda_fail(e, "write-back launch");
 }
 
 stq_status stq_pool_join(stq_pool *p, void *stream)

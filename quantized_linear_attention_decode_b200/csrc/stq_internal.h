@@ -13,6 +13,7 @@ namespace stq {
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kScaleBytes = 4 * kD; // fp32 scales at the start of a page
 constexpr int kPageAlign = 128;    // pages are padded to this many bytes
+constexpr size_t kStaticScratchFloats = size_t(1) << 20;  // built-in u~ buffer: 4 MiB, 8192 tiles
 
 // device error word bits
 constexpr uint32_t kErrIndex = 1u;

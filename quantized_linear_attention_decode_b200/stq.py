@@ -25,6 +25,7 @@ STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE
 EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
            "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
            "stq_decode_readout", "stq_decode_writeback", "stq_decode_step_split", "stq_pool_join",
+           "stq_decode_step_static",
            "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
            "stq_status_str", "stq_last_error")
 
@@ -68,6 +69,7 @@ def load():
         "stq_decode_writeback": [P, P, P, I32, P, P, P, P],
         "stq_decode_step_split": [P, P, P, I32, P, P, P, P, P, P, P, P, P],
         "stq_pool_join": [P, P],
+        "stq_decode_step_static": [P, P, P, I32, P, P, P, P, P, P, P],
         "stq_export_slot": [P, I32, I32, P, SZ],
         "stq_import_slot": [P, I32, I32, P, SZ],
         "stq_pool_check": [P, P],
@@ -258,6 +260,20 @@ def stq_decode_step_split(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y,
         pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
         _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
         _dev(u_tilde, f, vec, "u_tilde"), _stream(stream), _stream(side_stream)))
+
+
+def stq_decode_step_static(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, stream=None) -> None:
+    """stq_decode_step without any device allocation: u~ lives in the
+    library's built-in 4 MiB array (at most 8192 (entry, head) tiles per call;
+    calls that overlap on the GPU must be serialized by the caller)."""
+    import torch
+    n, r, s = _idx(pool, req_idx, slot_idx)
+    f = torch.float32
+    vec, gshape = _vecs(pool, n)
+    _check(load().stq_decode_step_static(
+        pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
+        _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
+        _stream(stream)))
 
 
 def stq_pool_join(pool: Pool, stream=None) -> None:
