@@ -226,6 +226,42 @@ stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const 
 /* Make `stream` wait for the pool's pending split write-back (no-op if none). */
 stq_status stq_pool_join(stq_pool *pool, void *stream);
 
+/*
+ * Lifetime-aware mixed-precision bit allocation (host computation; "core
+ * innovation", first point, and "method steps", offline calibration steps
+ * (1)-(3)).  Produces the unit_bits of a pool description from per-unit
+ * calibration statistics.
+ *
+ * stq_lifetime_weight: L_u = sum_{j=0}^{horizon-1} exp(2 j l_u) for each
+ *   unit's mean log retention l_u = E[log r_{t,u}] (<= 0): the factor by which
+ *   the squared error injected at one step is summed over the horizon.  The
+ *   page leaves the horizon open; it is an argument here.
+ * stq_allocate_bits: minimises sum_u L_u d_u(b_u) subject to
+ *   sum_u n_u b_u <= mean_bits * sum_u n_u (Eq. 8) over b_u in `choices`
+ *   (strictly increasing widths), with
+ *     unit_values n_u [U]   values per unit (a GDN head: 16384; a KDA row: 128),
+ *     distortion d_u(b) [U][C] (row-major, >= 0), weight L_u [U] (>= 0),
+ *     method STQ_ALLOC_DP       exact multiple-choice dynamic programme
+ *                               (integer n_u; STQ_ERR_UNSUPPORTED if the
+ *                               table would exceed 4e8 cells),
+ *            STQ_ALLOC_LAGRANGE per-unit minimiser of L d + lambda n b at the
+ *                               smallest multiplier that fits the budget
+ *                               (optimal for the bits it uses).
+ *   Afterwards the num_pivots units of largest remaining risk L_u d_u(b_u)
+ *   get pivot_bits (the page's FP16 pivots: 16); pivots are outside the
+ *   budget.  bits_out [U] receives the widths, objective_out (may be NULL)
+ *   the minimised sum before pivots.  Ties go to the smaller width.
+ *   STQ_ERR_ARG: bad sizes, non-finite or negative inputs, a budget below the
+ *   smallest width.
+ */
+typedef enum { STQ_ALLOC_DP = 0, STQ_ALLOC_LAGRANGE = 1 } stq_alloc_method;
+stq_status stq_lifetime_weight(int32_t num_units, const double *log_retention, int32_t horizon,
+                               double *weight_out);
+stq_status stq_allocate_bits(int32_t num_units, const double *unit_values, int32_t num_choices,
+                             const uint8_t *choices, const double *distortion, const double *weight,
+                             double mean_bits, int32_t method, int32_t num_pivots, uint8_t pivot_bits,
+                             uint8_t *bits_out, double *objective_out);
+
 /* Copy one slot's raw pages (per_slot_bytes bytes) to / from host memory.
  * Synchronous (device-wide ordering with the legacy default stream). */
 stq_status stq_export_slot(const stq_pool *pool, int32_t req, int32_t slot, void *host_dst,

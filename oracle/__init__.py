@@ -218,3 +218,33 @@ def near_tie(quot: np.ndarray, rel: float = 1e-4) -> np.ndarray:
     x = np.asarray(quot, np.float64)
     frac = np.abs(x - np.floor(x) - 0.5)
     return frac <= rel * np.maximum(np.abs(x), 1.0)
+
+
+# ---------------------------------------------------------------- bit allocation (pure Python, tiny cases)
+
+
+def lifetime_weight_sum(ell: float, horizon: int) -> float:
+    """L_u = sum_{j=0}^{H-1} exp(2 j l_u), term by term ("core innovation",
+    first point: an error's square decays by exp(2 l_u) per step)."""
+    import math
+    return math.fsum(math.exp(2.0 * j * ell) for j in range(horizon))
+
+
+def allocate_brute_force(unit_values, choices, distortion, weight, mean_bits, max_cost=None):
+    """Every assignment of widths to units (tiny instances only): the minimum
+    of sum_u L_u d_u(b_u) subject to sum_u n_u b_u <= mean_bits sum_u n_u
+    (Eq. 8), or <= max_cost when given.  Returns (objective, widths) of the
+    cheapest minimiser, or (inf, None) if nothing fits."""
+    import itertools
+    n = [float(x) for x in unit_values]
+    budget = mean_bits * sum(n) if max_cost is None else max_cost
+    best, best_cost, arg = float("inf"), float("inf"), None
+    for pick in itertools.product(range(len(choices)), repeat=len(n)):
+        cost = sum(n[u] * choices[k] for u, k in enumerate(pick))
+        if cost > budget * (1 + 1e-12):
+            continue
+        f = sum(weight[u] * distortion[u][k] for u, k in enumerate(pick))
+        if f < best or (f == best and cost < best_cost):
+            best, best_cost, arg = f, cost, [choices[k] for k in pick]
+    return best, arg
+

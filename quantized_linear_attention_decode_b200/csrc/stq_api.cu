@@ -236,6 +236,17 @@ stq_status check_split_args(const stq_pool *p, int32_t n, const float *u_tilde)
 
 namespace stq {
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+stq_status fail_status(stq_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
 }  // namespace stq
 
 using stq::kD;

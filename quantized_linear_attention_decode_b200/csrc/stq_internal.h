@@ -70,4 +70,7 @@ cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const i
 
 void count_launch();
 
+// Records a printf-style message for stq_last_error() and returns st.
+stq_status fail_status(stq_status st, const char *fmt, ...);
+
 }  // namespace stq

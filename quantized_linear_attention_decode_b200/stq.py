@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libstq.so")
 
 STQ_GDN, STQ_KDA = 0, 1
 STQ_SCALE_F16 = 1  # desc flag: per-row scales stored as IEEE binary16
+STQ_ALLOC_DP, STQ_ALLOC_LAGRANGE = 0, 1  # bit allocation methods
 STATUS = {0: "STQ_OK", 1: "STQ_ERR_ARG", 2: "STQ_ERR_OOM", 3: "STQ_ERR_CUDA", 4: "STQ_ERR_INDEX",
           5: "STQ_ERR_NONFINITE", 6: "STQ_ERR_UNSUPPORTED", 7: "STQ_ERR_TIMEOUT"}
 STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE, \
@@ -25,7 +26,7 @@ STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE
 EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
            "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
            "stq_decode_readout", "stq_decode_writeback", "stq_decode_step_split", "stq_pool_join",
-           "stq_decode_step_static",
+           "stq_decode_step_static", "stq_lifetime_weight", "stq_allocate_bits",
            "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
            "stq_status_str", "stq_last_error")
 
@@ -70,6 +71,8 @@ def load():
         "stq_decode_step_split": [P, P, P, I32, P, P, P, P, P, P, P, P, P],
         "stq_pool_join": [P, P],
         "stq_decode_step_static": [P, P, P, I32, P, P, P, P, P, P, P],
+        "stq_lifetime_weight": [I32, P, I32, P],
+        "stq_allocate_bits": [I32, P, I32, P, P, P, C.c_double, I32, I32, C.c_uint8, P, P],
         "stq_export_slot": [P, I32, I32, P, SZ],
         "stq_import_slot": [P, I32, I32, P, SZ],
         "stq_pool_check": [P, P],
@@ -274,6 +277,30 @@ def stq_decode_step_static(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y
         pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
         _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
         _stream(stream)))
+
+
+def stq_lifetime_weight(log_retention, horizon: int) -> np.ndarray:
+    """L_u = sum_{j < horizon} exp(2 j l_u) for each unit's mean log retention."""
+    ell = np.ascontiguousarray(log_retention, np.float64).reshape(-1)
+    out = np.empty_like(ell)
+    _check(load().stq_lifetime_weight(len(ell), ell.ctypes.data, int(horizon), out.ctypes.data))
+    return out
+
+
+def stq_allocate_bits(unit_values, choices, distortion, weight, mean_bits: float, method: int = STQ_ALLOC_DP,
+                      num_pivots: int = 0, pivot_bits: int = 16):
+    """Per-unit widths minimising sum L_u d_u(b_u) under the mean-bits budget
+    (then the num_pivots riskiest units at pivot_bits); returns (bits, objective)."""
+    n = np.ascontiguousarray(unit_values, np.float64).reshape(-1)
+    ch = np.ascontiguousarray(choices, np.uint8).reshape(-1)
+    d = np.ascontiguousarray(distortion, np.float64).reshape(len(n), len(ch))
+    w = np.ascontiguousarray(weight, np.float64).reshape(len(n))
+    bits = np.zeros(len(n), np.uint8)
+    obj = C.c_double()
+    _check(load().stq_allocate_bits(len(n), n.ctypes.data, len(ch), ch.ctypes.data, d.ctypes.data, w.ctypes.data,
+                                    float(mean_bits), int(method), int(num_pivots), int(pivot_bits),
+                                    bits.ctypes.data, C.byref(obj)))
+    return bits, obj.value
 
 
 def stq_pool_join(pool: Pool, stream=None) -> None:
