@@ -85,13 +85,15 @@ def _f64(a):
     return np.ascontiguousarray(a, dtype=np.float64)
 
 
-# scale formats: fp32 scales (0), IEEE binary16 scales (1).  Units whose rows
-# are all 16 or all 32 bits wide are raw (binary16 / binary32 values, no scales).
-FMT_F32, FMT_F16 = 0, 1
+# scale formats: fp32 scales (0), IEEE binary16 scales (1); flag FMT_PIVOT (4):
+# 16-bit rows are FP16 pivots among quantized rows (scale slot 1, binary16
+# mu = X / (r c)).  Without the flag, units whose rows are all 16 or all 32
+# bits wide are raw (binary16 / binary32 values, no scales).
+FMT_F32, FMT_F16, FMT_PIVOT = 0, 1, 4
 
 
-def is_raw(bits) -> bool:
-    return int(np.asarray(bits).reshape(-1)[0]) in (16, 32)
+def is_raw(bits, fmt: int = FMT_F32) -> bool:
+    return not (fmt & FMT_PIVOT) and int(np.asarray(bits).reshape(-1)[0]) in (16, 32)
 
 
 def page_bytes(bits, dv: int | None = None, fmt: int = FMT_F32) -> int:
@@ -105,7 +107,7 @@ def row_offsets(bits, dv: int | None = None, fmt: int = FMT_F32) -> np.ndarray:
     bits = np.asarray(bits, dtype=np.int64)
     dv = len(bits) if dv is None else dv
     sizes = dv * bits // 8
-    sb = 0 if is_raw(bits) else (2 if fmt == FMT_F16 else 4)
+    sb = 0 if is_raw(bits, fmt) else (2 if fmt & FMT_F16 else 4)
     return sb * len(bits) + np.concatenate([[0], np.cumsum(sizes)[:-1]])
 
 

@@ -36,10 +36,17 @@
  *     binary16, s16 = half(a_i / q_b) rounded to nearest even, and the codes
  *     are then rounded from mu_ij / s16 so that s16 z reconstructs them; a
  *     scale above the binary16 range is reported like a non-finite row;
- *   - raw units ("FP16 pivot units" and the fp32 control state): every row
- *     of the unit is 16 or 32 bits wide and holds the state value itself in
- *     IEEE binary16 / binary32, with no scale and no r, c factors; the step is
- *     the same recurrence, and X is rounded once (to nearest even) on store;
+ *   - raw units (the page's FP16 storage applied to a whole pool, and the
+ *     fp32 control state): every row of the unit is 16 or 32 bits wide and
+ *     holds the state value itself in IEEE binary16 / binary32, with no scale
+ *     and no r, c factors; the step is the same recurrence, and X is rounded
+ *     once (to nearest even) on store;
+ *   - FP16 pivots ([steps] step 1: "pivot units are read in FP16 directly";
+ *     format flag 4, a pool that mixes pivots with quantized units): a
+ *     16-bit row keeps its scale slot, which holds 1, and stores
+ *     mu_ij = fl32(X_ij / (r_i c_j)) rounded once to binary16 in place of
+ *     the codes; it reconstructs as s_i r_i c_j mu_ij like a quantized row
+ *     (with r = c = 1, the state value itself);
  *   - the continuous part (reconstruction, decay, retrieval, write,
  *     readout) is computed in fp64; the quantisation decision is taken in
  *     fp32 on the fp32-rounded value mu_ij = fl32(X_ij / (r_i c_j)), with
@@ -72,22 +79,30 @@ static int q_of_bits(int b) { return (1 << (b - 1)) - 1; }
 
 static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8u; }
 
+/* format flags: bit 0 binary16 scales, bit 2 FP16 pivot rows among quantized ones */
+#define ORC_FMT_F16 1
+#define ORC_FMT_PIVOT 4
+
+static int fmt_ok(int fmt) { return fmt >= 0 && (fmt & ~(ORC_FMT_F16 | ORC_FMT_PIVOT)) == 0; }
+
 /* 16 or 32 for a raw unit (its first row decides; bits_ok checks the rest), else 0 */
-static int raw_width(int dk, const uint8_t *bits)
+static int raw_width(int dk, const uint8_t *bits, int fmt)
 {
-    if (dk <= 0) return 0;
+    if (dk <= 0 || (fmt & ORC_FMT_PIVOT)) return 0;
     return (bits[0] == 16 || bits[0] == 32) ? bits[0] : 0;
 }
 
-/* quantized rows are 4, 6 or 8 bits; a raw unit has all rows at 16 or at 32 */
-static int bits_ok(int dk, int dv, const uint8_t *bits)
+/* quantized rows are 4, 6 or 8 bits (or 16, pivots, under ORC_FMT_PIVOT); a raw
+ * unit has all rows at 16 or at 32 */
+static int bits_ok(int dk, int dv, const uint8_t *bits, int fmt)
 {
-    int raw = raw_width(dk, bits);
+    if (!fmt_ok(fmt)) return 0;
+    int raw = raw_width(dk, bits, fmt);
     for (int i = 0; i < dk; ++i) {
         int b = bits[i];
         if (raw) {
             if (b != raw) return 0;
-        } else if (b != 4 && b != 6 && b != 8) {
+        } else if (b != 4 && b != 6 && b != 8 && !(b == 16 && (fmt & ORC_FMT_PIVOT))) {
             return 0;
         }
         if ((dv * b) % 8 != 0) return 0;
@@ -95,11 +110,11 @@ static int bits_ok(int dk, int dv, const uint8_t *bits)
     return 1;
 }
 
-/* bytes per scale: fmt 0 fp32, fmt 1 binary16; a raw unit has none */
+/* bytes per scale: fp32, or binary16 with ORC_FMT_F16; a raw unit has none */
 static size_t scale_bytes(int dk, const uint8_t *bits, int fmt)
 {
-    if (raw_width(dk, bits)) return 0;
-    return fmt == 1 ? 2u : 4u;
+    if (raw_width(dk, bits, fmt)) return 0;
+    return (fmt & ORC_FMT_F16) ? 2u : 4u;
 }
 
 size_t orc_page_bytes_fmt(int dk, int dv, const uint8_t *bits, int fmt)
@@ -180,7 +195,7 @@ static void put_code(uint8_t *row, int b, int j, int32_t z)
 
 static float get_scale(const uint8_t *page, int fmt, int i)
 {
-    if (fmt == 1) {
+    if (fmt & ORC_FMT_F16) {
         uint16_t h;
         memcpy(&h, page + 2 * (size_t)i, 2);
         return (float)orc_half_to_double(h);
@@ -193,7 +208,7 @@ static float get_scale(const uint8_t *page, int fmt, int i)
 /* stores s (format 0) or half(s) (format 1); returns the value stored, as a float */
 static float put_scale(uint8_t *page, int fmt, int i, float s)
 {
-    if (fmt == 1) {
+    if (fmt & ORC_FMT_F16) {
         uint16_t h = orc_double_to_half((double)s);
         memcpy(page + 2 * (size_t)i, &h, 2);
         return (float)orc_half_to_double(h);
@@ -232,11 +247,12 @@ static double put_raw(uint8_t *row, int b, int j, double x)
 int32_t orc_get_code(const uint8_t *row, int b, int j) { return get_code(row, b, j); }
 void orc_put_code(uint8_t *row, int b, int j, int32_t z) { put_code(row, b, j, z); }
 
-/* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 (a raw unit: the stored value) */
+/* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 (a raw unit: the stored
+ * value; a pivot row: z_ij is its binary16 value) */
 static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                         int fmt, const uint8_t *page, double *S)
 {
-    int raw = raw_width(dk, bits);
+    int raw = raw_width(dk, bits, fmt);
     for (int i = 0; i < dk; ++i) {
         const uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
         if (raw) {
@@ -245,8 +261,8 @@ static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, con
         }
         double s = (double)get_scale(page, fmt, i);
         for (int j = 0; j < dv; ++j) {
-            int32_t z = get_code(row, bits[i], j);
-            S[(size_t)i * dv + j] = s * (double)r[i] * (double)c[j] * (double)z;
+            double z = bits[i] == 16 ? get_raw(row, 16, j) : (double)get_code(row, bits[i], j);
+            S[(size_t)i * dv + j] = s * (double)r[i] * (double)c[j] * z;
         }
     }
 }
@@ -261,7 +277,7 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
                       int fmt, const double *X, uint8_t *page, float *quot)
 {
     int status = ORC_OK;
-    int raw = raw_width(dk, bits);
+    int raw = raw_width(dk, bits, fmt);
     if (raw) {
         /* raw unit: X rounded once to the row format; quot receives fl32(X) */
         for (int i = 0; i < dk; ++i) {
@@ -277,6 +293,19 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
     }
     float *mu = (float *)malloc(sizeof(float) * (size_t)dv);
     for (int i = 0; i < dk; ++i) {
+        if (bits[i] == 16) {
+            /* pivot row: scale slot 1, mu rounded once to binary16; quot receives mu */
+            uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
+            put_scale(page, fmt, i, 1.0f);
+            for (int j = 0; j < dv; ++j) {
+                double rc = (double)r[i] * (double)c[j];
+                float m = (float)(X[(size_t)i * dv + j] / rc);
+                double st = put_raw(row, 16, j, (double)m);
+                if (!isfinite(st)) status = ORC_NONFINITE;
+                if (quot) quot[(size_t)i * dv + j] = m;
+            }
+            continue;
+        }
         int qb = q_of_bits(bits[i]);
         float a = 0.0f;
         for (int j = 0; j < dv; ++j) {
@@ -311,7 +340,7 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
 int orc_quantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                           int fmt, const float *S, uint8_t *page, float *quot)
 {
-    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
+    if (!bits_ok(dk, dv, bits, fmt)) return ORC_BADARG;
     size_t nb = orc_page_bytes_fmt(dk, dv, bits, fmt);
     memset(page, 0, nb);
     double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
@@ -331,7 +360,7 @@ int orc_quantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const
 int orc_dequantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
                             int fmt, const uint8_t *page, float *S)
 {
-    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
+    if (!bits_ok(dk, dv, bits, fmt)) return ORC_BADARG;
     double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
     reconstruct(dk, dv, bits, r, c, fmt, page, X);
     for (size_t e = 0; e < (size_t)dk * dv; ++e) S[e] = (float)X[e];
@@ -362,7 +391,7 @@ int orc_step_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const
                       const float *q, const float *k, const float *v, float beta, const float *g,
                       double *y, float *quot)
 {
-    if (!bits_ok(dk, dv, bits) || fmt < 0 || fmt > 1) return ORC_BADARG;
+    if (!bits_ok(dk, dv, bits, fmt)) return ORC_BADARG;
     size_t nel = (size_t)dk * dv;
     double *P = (double *)malloc(sizeof(double) * nel);
     double *vo = (double *)malloc(sizeof(double) * (size_t)dv);

@@ -189,3 +189,126 @@ def test_raw_units_must_be_uniform():
     bits[3] = 8
     with pytest.raises(ValueError):
         orc.quantize_unit(bits, np.ones(D), np.ones(D), np.zeros((D, D), np.float32))
+
+
+# ---------------------------------------------------------------- FP16 pivot rows among quantized rows
+
+
+PIV = orc.FMT_PIVOT
+
+
+def _pivot_values(page, bits, dv, fmt):
+    offs = orc.row_offsets(bits, dv, fmt)
+    out = np.full((len(bits), dv), np.nan)
+    for i, b in enumerate(bits):
+        if b == 16:
+            out[i] = page[offs[i]: offs[i] + 2 * dv].view(np.float16).astype(np.float64)
+    return out
+
+
+@pytest.mark.parametrize("fmt", [PIV, PIV | orc.FMT_F16])
+def test_pivot_rows_round_trip_exactly_and_leave_other_rows_alone(fmt):
+    """Values representable in binary16 come back exactly from pivot rows (scale slot 1);
+    the quantized rows are byte-identical to the same rows quantized without pivots."""
+    rng = RNG(40)
+    bits = np.array([6, 16, 8, 4, 16, 6, 8, 16], np.uint8)
+    S = rng.standard_normal((D, D)).astype(np.float16).astype(np.float32)
+    ones = np.ones(D, np.float32)
+    page = orc.quantize_unit(bits, ones, ones, S, fmt=fmt)
+    assert len(page) == orc.page_bytes(bits, D, fmt)
+    back = orc.dequantize_unit(bits, ones, ones, page, D, fmt)
+    piv = bits == 16
+    np.testing.assert_array_equal(back[piv], S[piv])
+    sc = page[: 2 * D].view(np.float16).astype(np.float32) if fmt & orc.FMT_F16 else page[: 4 * D].view(np.float32)
+    np.testing.assert_array_equal(sc[piv], 1.0)
+    alt = bits.copy()
+    alt[piv] = 8
+    ref = orc.quantize_unit(alt, ones, ones, S, fmt=fmt & orc.FMT_F16)
+    offs, offs_alt = orc.row_offsets(bits, D, fmt), orc.row_offsets(alt, D, fmt & orc.FMT_F16)
+    for i in np.nonzero(~piv)[0]:
+        n = D * int(bits[i]) // 8
+        assert page[offs[i]: offs[i] + n].tobytes() == ref[offs_alt[i]: offs_alt[i] + n].tobytes()
+    np.testing.assert_array_equal(sc[~piv], (ref[: 2 * D].view(np.float16).astype(np.float32)
+                                            if fmt & orc.FMT_F16 else ref[: 4 * D].view(np.float32))[~piv])
+
+
+def test_pivot_rows_hold_the_binary16_state_over_the_factors():
+    """With r, c != 1 a pivot row stores half(fl32(X / (r c))): the rank-one first step
+    from zero, X = beta k v^T, checked element by element with numpy's binary16."""
+    rng = RNG(41)
+    bits = np.array([16, 6, 16, 8, 16, 4, 6, 16], np.uint8)
+    r = np.exp(rng.uniform(-1, 1, D)).astype(np.float32)
+    c = np.exp(rng.uniform(-1, 1, D)).astype(np.float32)
+    page0 = orc.quantize_unit(bits, r, c, np.zeros((D, D), np.float32), fmt=PIV)
+    k, q = _unit(D, rng), _unit(D, rng)
+    v = rng.standard_normal(D).astype(np.float32)
+    beta = np.float32(0.7)
+    out, y, quot, st = orc.step_unit(bits, r, c, page0, q, k, v, beta, np.full(D, 0.9, np.float32), D, PIV)
+    assert st == orc.OK
+    X = float(beta) * np.outer(k.astype(np.float64), v.astype(np.float64))
+    mu = (X / np.outer(r.astype(np.float64), c.astype(np.float64))).astype(np.float32)
+    got = _pivot_values(out, bits, D, PIV)
+    piv = bits == 16
+    np.testing.assert_array_equal(got[piv], mu[piv].astype(np.float16).astype(np.float64))
+    np.testing.assert_allclose(y, X.T @ q.astype(np.float64), rtol=1e-12, atol=1e-15)
+
+
+def test_pivot_unit_equals_raw16_unit_when_factors_are_one():
+    """A head made only of pivot rows (r = c = 1) takes the raw binary16 unit's step:
+    same readout, same stored values."""
+    rng = RNG(42)
+    bits = np.full(D, 16, np.uint8)
+    ones = np.ones(D, np.float32)
+    S = rng.standard_normal((D, D)).astype(np.float32)
+    p_piv = orc.quantize_unit(bits, ones, ones, S, fmt=PIV)
+    p_raw = orc.quantize_unit(bits, ones, ones, S)
+    for t in range(4):
+        q, k = _unit(D, rng), _unit(D, rng)
+        v = rng.standard_normal(D).astype(np.float32)
+        g = rng.uniform(0.8, 1.0, D).astype(np.float32)
+        p_piv, y1, _, s1 = orc.step_unit(bits, ones, ones, p_piv, q, k, v, np.float32(0.6), g, D, PIV)
+        p_raw, y2, _, s2 = orc.step_unit(bits, ones, ones, p_raw, q, k, v, np.float32(0.6), g, D)
+        assert s1 == s2 == orc.OK
+        np.testing.assert_array_equal(y1, y2)
+        np.testing.assert_array_equal(_pivot_values(p_piv, bits, D, PIV), _raw_values(p_raw, bits, D))
+
+
+def test_pivot_step_is_the_rounded_explicit_recurrence():
+    """Mixed unit: the pivot rows of the next page are the explicit recurrence (fp64, on
+    the reconstructed state) over r c, rounded to fp32 then binary16; the readout is
+    the explicit readout."""
+    rng = RNG(43)
+    bits = np.array([6, 16, 8, 16, 4, 6, 16, 8], np.uint8)
+    r = np.exp(rng.uniform(-0.5, 0.5, D)).astype(np.float32)
+    c = np.exp(rng.uniform(-0.5, 0.5, D)).astype(np.float32)
+    page = orc.quantize_unit(bits, r, c, rng.standard_normal((D, D)).astype(np.float32), fmt=PIV)
+    q, k = _unit(D, rng), _unit(D, rng)
+    v = rng.standard_normal(D).astype(np.float32)
+    g = rng.uniform(0.8, 1.0, D).astype(np.float32)
+    S_hat = orc.dequantize_unit(bits, r, c, page, D, PIV).astype(np.float64)
+    # the reconstruction itself, recomputed from the stored values
+    Sv = _pivot_values(page, bits, D, PIV)
+    piv = bits == 16
+    np.testing.assert_array_equal(S_hat[piv], (np.outer(r.astype(np.float64), c.astype(np.float64)) * Sv)[piv].astype(np.float32))
+    exact = np.outer(r.astype(np.float64), c.astype(np.float64)) * np.where(np.isnan(Sv), 0, Sv)
+    exact[~piv] = S_hat[~piv]
+    out, y, _, st = orc.step_unit(bits, r, c, page, q, k, v, np.float32(0.8), g, D, PIV)
+    X, y_ref = _explicit_step(exact, q, k, v, 0.8, g)
+    np.testing.assert_allclose(y, y_ref, rtol=1e-6, atol=1e-6 * np.abs(y_ref).max())
+    mu = (X / np.outer(r.astype(np.float64), c.astype(np.float64))).astype(np.float32).astype(np.float16)
+    got = _pivot_values(out, bits, D, PIV)
+    # the explicit form and the oracle's delta form agree to fp64 rounding; both then round
+    # to binary16, which can differ by one step only next to a rounding midpoint
+    d = np.abs(got[piv] - mu[piv].astype(np.float64))
+    spacing = np.abs(np.spacing(mu[piv])).astype(np.float64)
+    assert np.all(d <= spacing)
+    assert np.count_nonzero(d) <= 1
+
+
+def test_pivot_rows_need_the_flag_and_reject_32():
+    ones = np.ones(D, np.float32)
+    S = np.zeros((D, D), np.float32)
+    with pytest.raises(ValueError):
+        orc.quantize_unit(np.array([6, 16, 6, 6, 6, 6, 6, 6], np.uint8), ones, ones, S)
+    with pytest.raises(ValueError):
+        orc.quantize_unit(np.array([6, 32, 6, 6, 6, 6, 6, 6], np.uint8), ones, ones, S, fmt=PIV)
