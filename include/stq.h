@@ -63,11 +63,17 @@ typedef struct stq_pool stq_pool;
  * Pool description ("SGLang state pool" section: pool = concurrency x slots
  * x per-request state).  A unit of precision ("core method" section: a whole
  * head for GDN, one key row for KDA) carries a bit width b in {4, 6, 8}
- * (quantized codes).  Raw pools hold the state values themselves: every unit
- * at 16 (IEEE binary16, the page's FP16 "pivot" storage applied to the whole
- * pool) or every unit at 32 (fp32, the unquantized control the page's
- * state-update timings compare against); mixing raw and quantized units in
- * one pool returns STQ_ERR_UNSUPPORTED.
+ * (quantized codes) or 16: an FP16 pivot unit ("method steps", step 1, and
+ * offline step (3): the riskiest units are kept in FP16, 32 of 2304 GDN heads
+ * and 512 of 81920 KDA rows in the page's setting).  A pivot row keeps its
+ * scale slot, which holds 1, and stores mu_ij = X_ij / (r_i c_j) rounded once
+ * to binary16 (the state itself when r = c = 1).  A KDA head's page must stay
+ * within 16896 bytes (pivot rows averaging at most 8 bits per row over the
+ * head), else STQ_ERR_UNSUPPORTED.
+ * Raw pools hold the state values themselves: every unit at 16 (IEEE
+ * binary16, no scales, r and c unused) or every unit at 32 (fp32, the
+ * unquantized control the page's state-update timings compare against); fp32
+ * units mixed with others return STQ_ERR_UNSUPPORTED.
  */
 #define STQ_SCALE_F16 1u /* flags: per-row scales stored as IEEE binary16 ("method steps", step 6) */
 
@@ -183,6 +189,8 @@ stq_status stq_decode_step(stq_pool *pool, const int32_t *req_idx, const int32_t
  *                       given stream wait for it.  Before capturing a CUDA
  *                       graph, join or synchronize any write-back issued
  *                       outside the capture.
+ * GDN pivot heads are advanced completely by the readout (their own kernel
+ * stores the new binary16 values); every other unit as described.
  * Raw pools (units of 16 or 32 bits) return STQ_ERR_UNSUPPORTED.  Argument
  * rules are those of stq_decode_step; u_tilde must not be NULL for n > 0.
  */

@@ -16,6 +16,8 @@
 struct stq_pool {
     int kind = 0, R = 0, S = 0, H = 0;
     int scale_bytes = 4, raw_bits = 0;
+    bool pivots = false;       // FP16 pivot units among quantized ones
+    bool pivot_heads = false;  // GDN pivot heads (their own kernel)
     int device = 0;
     size_t slot_bytes = 0, packed_bytes = 0;
     uint8_t *d_pages = nullptr;
@@ -75,11 +77,21 @@ HeadLayout head_layout(const uint8_t *row_bits, int scale_bytes)
     return L;
 }
 
+// Width of a raw pool (every unit 16, or every unit 32 bits), else 0.
+int raw_width_of(const stq_pool_desc *d)
+{
+    const size_t nunits = d->kind == STQ_GDN ? (size_t)d->num_heads : (size_t)d->num_heads * stq::kD;
+    const int b0 = d->unit_bits[0];
+    if (b0 != 16 && b0 != 32) return 0;
+    for (size_t u = 1; u < nunits; ++u)
+        if (d->unit_bits[u] != b0) return 0;
+    return b0;
+}
+
 // Bytes per row scale of a (validated) description: 0 for a raw pool.
 int scale_bytes_of(const stq_pool_desc *d)
 {
-    const int b0 = d->unit_bits[0];
-    if (b0 == 16 || b0 == 32) return 0;
+    if (raw_width_of(d)) return 0;
     return (d->flags & STQ_SCALE_F16) ? 2 : 4;
 }
 
@@ -97,16 +109,16 @@ stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
     const int H = d->num_heads;
     const size_t nunits = d->kind == STQ_GDN ? (size_t)H : (size_t)H * stq::kD;
     if (d->flags & ~STQ_SCALE_F16) return fail(STQ_ERR_ARG, "flags 0x%x", d->flags);
-    const int b0 = d->unit_bits[0];
-    const bool raw = b0 == 16 || b0 == 32;
     for (size_t u = 0; u < nunits; ++u) {
         int b = d->unit_bits[u];
         if (b != 4 && b != 6 && b != 8 && b != 16 && b != 32)
             return fail(STQ_ERR_ARG, "unit_bits[%zu] = %d (must be 4, 6, 8, 16 or 32)", u, b);
-        if (raw ? b != b0 : (b == 16 || b == 32))
-            return fail(STQ_ERR_UNSUPPORTED, "unit_bits[%zu] = %d: raw (16 / 32-bit) units must make up "
-                        "the whole pool, at one width", u, b);
     }
+    const int raw = raw_width_of(d);
+    if (!raw)
+        for (size_t u = 0; u < nunits; ++u)
+            if (d->unit_bits[u] == 32)
+                return fail(STQ_ERR_UNSUPPORTED, "unit_bits[%zu] = 32: fp32 units must make up the whole pool", u);
     if (raw && d->flags != 0) return fail(STQ_ERR_ARG, "a raw pool has no scales (flags must be 0)");
     for (int which = 0; which < 2; ++which) {
         const float *f = which ? d->col_factor : d->row_factor;
@@ -134,6 +146,9 @@ stq_status sizes_of(const stq_pool_desc *d, const std::vector<uint8_t> &row_bits
     const int sb = scale_bytes_of(d);
     for (int h = 0; h < d->num_heads; ++h) {
         HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD], sb);
+        if (d->kind == STQ_KDA && sb != 0 && L.page_bytes > (uint32_t)stq::kMaxStagedPage)
+            return fail(STQ_ERR_UNSUPPORTED, "KDA head %d: %u-byte page (FP16 pivot rows average above 8 bits "
+                        "per row); at most %d bytes", h, L.page_bytes, stq::kMaxStagedPage);
         if (head_off) head_off->push_back((uint32_t)off);
         if (page_bytes) page_bytes->push_back(L.page_bytes);
         off += L.page_bytes;
@@ -157,6 +172,7 @@ stq::PoolView view(stq_pool *p)
     v.kind = p->kind;
     v.scale_bytes = p->scale_bytes;
     v.raw_bits = p->raw_bits;
+    v.pivots = p->pivots ? 1 : 0;
     v.t = p->t;
     v.err = p->d_err;
     return v;
@@ -300,7 +316,9 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->S = desc->num_slots;
     p->H = desc->num_heads;
     p->scale_bytes = scale_bytes_of(desc);
-    p->raw_bits = p->scale_bytes == 0 ? desc->unit_bits[0] : 0;
+    p->raw_bits = raw_width_of(desc);
+    for (size_t u = 0; !p->raw_bits && u < rb.size(); ++u) p->pivots |= rb[u] == 16;
+    p->pivot_heads = p->pivots && p->kind == STQ_GDN;
     st = sizes_of(desc, rb, &p->head_off, &p->page_bytes, &p->slot_bytes, &p->packed_bytes);
     if (st != STQ_OK) {
         delete p;
@@ -333,11 +351,11 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
         uint8_t *blk = &img[o_blk + (size_t)h * stq::kHeadBlock];
         std::memcpy(blk, fr + (size_t)h * kD, kD * 4);
         std::memcpy(blk + 512, fc + (size_t)h * kD, kD * 4);
-        float inv_rq[kD];  // 1 / (r_i q_b(i)), rounded once from double (unused by raw pages)
+        float inv_rq[kD];  // 1 / (r_i q_b(i)), rounded once from double; 1 / r_i for a pivot row (unused by raw pages)
         for (int i = 0; i < kD; ++i) {
             const int b = rb[(size_t)h * kD + i];
-            inv_rq[i] = b <= 8 ? (float)(1.0 / ((double)fr[(size_t)h * kD + i] * (double)((1 << (b - 1)) - 1)))
-                               : 0.0f;
+            const double r = (double)fr[(size_t)h * kD + i];
+            inv_rq[i] = b <= 8 ? (float)(1.0 / (r * (double)((1 << (b - 1)) - 1))) : b == 16 ? (float)(1.0 / r) : 0.0f;
         }
         std::memcpy(blk + 1024, inv_rq, kD * 4);
         std::memcpy(blk + 1536, &img[o_ro + (size_t)h * kD * 2], kD * 2);
@@ -458,6 +476,7 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, nullptr};
     e = p->raw_bits ? stq::launch_decode_raw(view(p), io, (cudaStream_t)stream)
                     : stq::launch_decode(view(p), io, (cudaStream_t)stream);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "decode launch");
 }
 
@@ -478,6 +497,7 @@ stq_status stq_decode_readout(stq_pool *p, const int32_t *req_idx, const int32_t
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u_tilde};
     e = stq::launch_decode_readout(view(p), io, (cudaStream_t)stream);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "readout launch");
 }
 
@@ -527,6 +547,7 @@ stq_status stq_decode_step_split(stq_pool *p, const int32_t *req_idx, const int3
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u_tilde};
     e = stq::launch_decode_readout(view(p), io, s0);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
     if (e != cudaSuccess) return cuda_fail(e, "readout launch");
     e = cudaEventRecord(p->ev_read, s0);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(s1, p->ev_read, 0);
@@ -605,6 +626,7 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
     // the readout fills u~ for every tile of the call before the write-back reads it
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u};
     e = stq::launch_decode_readout(view(p), io, s0);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
     if (e != cudaSuccess) return cuda_fail(e, "readout launch");
     stq::DecodeIO wb{req_idx, slot_idx, n, nullptr, k, u, nullptr, gate, nullptr, nullptr};
     e = stq::launch_decode_writeback(view(p), wb, s0);

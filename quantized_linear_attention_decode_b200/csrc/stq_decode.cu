@@ -48,7 +48,7 @@ constexpr int kFused = 0;      // the whole step (one state traversal)
 constexpr int kReadout = 1;    // steps 1-3: y and u~; the page is only read
 constexpr int kWriteback = 2;  // steps 4-7 given u~: requantise and pack in place
 constexpr int kStages = 4;
-constexpr int kMaxPage = kScaleBytes + 16 * 8 * kD;    // 16896: every row at 8 bits
+constexpr int kMaxPage = kMaxStagedPage;               // 16896: every row at 8 bits
 constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
 
 struct __align__(128) Stage {
@@ -353,9 +353,38 @@ template <> struct Codec<6> {
     }
 };
 
+// FP16 pivot rows ("method steps", step 1: pivot units are read in FP16
+// directly): the row holds mu = X / (r c) as 128 binary16 values; a thread's 8
+// columns are one 16-byte vector.  The scale slot of the row holds 1, so the
+// row enters both passes like a quantized row whose codes are mu.
+struct Pivot16 {
+    __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
+    {
+        const uint4 w = *reinterpret_cast<const uint4 *>(rowp + cg * 16);
+        z[0] = __half22float2(*reinterpret_cast<const __half2 *>(&w.x));
+        z[1] = __half22float2(*reinterpret_cast<const __half2 *>(&w.y));
+        z[2] = __half22float2(*reinterpret_cast<const __half2 *>(&w.z));
+        z[3] = __half22float2(*reinterpret_cast<const __half2 *>(&w.w));
+    }
+    // t: the new mu of the 8 columns, rounded once to binary16 (nearest even)
+    __device__ __forceinline__ static void store(uint8_t *rowg, int cg, const float2 t[4])
+    {
+        __half2 h[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) h[p] = __float22half2_rn(t[p]);
+        uint4 w;
+        w.x = *reinterpret_cast<const uint32_t *>(&h[0]);
+        w.y = *reinterpret_cast<const uint32_t *>(&h[1]);
+        w.z = *reinterpret_cast<const uint32_t *>(&h[2]);
+        w.w = *reinterpret_cast<const uint32_t *>(&h[3]);
+        *reinterpret_cast<uint4 *>(rowg + cg * 16) = w;
+    }
+};
+
 __device__ __forceinline__ void unpack_any(int b, const uint8_t *rowp, int cg, float2 z[4])
 {
-    if (b == 8) Codec<8>::unpack(rowp, cg, z);
+    if (b == 16) Pivot16::unpack(rowp, cg, z);
+    else if (b == 8) Codec<8>::unpack(rowp, cg, z);
     else if (b == 6) Codec<6>::unpack(rowp, cg, z);
     else Codec<4>::unpack(rowp, cg, z);
 }
@@ -569,7 +598,12 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
             const float qb = static_cast<float>((1 << (b - 1)) - 1);
             const float mrq = R.mrq[i];
             float inv = 0.0f, snew = 0.0f;
-            if (SB == 4) {
+            if (B == 0 && b == 16) {
+                // pivot row: the scale slot keeps 1; mu beyond the binary16 range is reported
+                if (!(fabsf(mrq) * m < 65520.0f)) atomicOr(&sm.flags, kErrNonFinite);
+                if (SB == 4) reinterpret_cast<float *>(page)[i] = 1.0f;
+                else reinterpret_cast<__half *>(page)[i] = __float2half_rn(1.0f);
+            } else if (SB == 4) {
                 if (m >= 1e-30f && m <= 3.0e38f) {
                     inv = copysignf(qb * rcp_approx(m), mrq);
                     snew = fabsf(mrq) * m;
@@ -607,6 +641,15 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
         const int b = B != 0 ? B : R.bits[i];
+        if (B == 0 && b == 16) {
+            // pivot row: mu = X / (r c) = (e / r) w, with R.mrq = e / r for a pivot row
+            const float2 m2 = make_float2(R.mrq[i], R.mrq[i]);
+            float2 t[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) t[p] = fmul2(z[ii][p], m2);
+            Pivot16::store(page + R.off[i], cg, t);
+            continue;
+        }
         const float mg = B != 0 ? Codec<B == 0 ? 8 : B>::kMagicOut : magic_out(b);
         const float2 inv2 = make_float2(invs[ii], invs[ii]), mg2 = make_float2(mg, mg);
         uint32_t bits[8];
@@ -670,9 +713,11 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
 {
     Stage &S = sm.st[s];
     sm.stage_page[s] = t.page;
-    sm.stage_valid[s] = t.valid;
-    if (!t.valid) {
-        atomicOr(&sm.flags, kErrIndex);
+    // a page larger than a stage is a GDN FP16 pivot head, advanced by its own kernel
+    const bool mine = t.valid && t.bytes <= static_cast<uint32_t>(kMaxPage);
+    sm.stage_valid[s] = mine;
+    if (!mine) {
+        if (!t.valid) atomicOr(&sm.flags, kErrIndex);
         mbar_arrive(&sm.full[s]);  // completes the phase with no data; the tile is skipped
         return;
     }
@@ -818,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         float2 z[8][4];
         constexpr bool kAcc = MODE != kWriteback;
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0, SB, kAcc>(sm, S, R, z);
+            if (KIND == STQ_KDA) pass1<0, SB, kAcc>(sm, S, R, z);  // per-row widths (and KDA pivot rows)
             else if (b == 8) pass1<8, SB, kAcc>(sm, S, R, z);
             else if (b == 6) pass1<6, SB, kAcc>(sm, S, R, z);
             else pass1<4, SB, kAcc>(sm, S, R, z);

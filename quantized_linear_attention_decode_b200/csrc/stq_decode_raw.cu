@@ -9,6 +9,13 @@
 //   P = D S,  u = beta (v - P^T k),  X = P + k u^T,  y = X^T q,  S <- round(X).
 // y = P^T q + (k.q) u, so one pass over S forms both column sums.
 //
+// The same kernel advances the GDN FP16 pivot heads of a quantized pool
+// (PIVOT): their page keeps the pool's scale section (slots of 1) and stores
+// mu = X / (r c) in binary16, so with P = g S and S_ij = r_i c_j mu_ij
+//   column sums over (g k r)_i mu_ij and (g q r)_i mu_ij, times c_j;
+//   mu'_ij = g mu_ij + (k_i / r_i) (u_j / c_j).
+// CTAs of the other heads return at once.
+//
 // One CTA (256 threads) per (request, head) tile.  Thread (rg, cg) = (2 warp +
 // lane / 16, lane % 16) holds rows [8 rg, 8 rg + 8) x columns [8 cg, 8 cg + 8)
 // in registers between the two passes; a half-warp reads or writes one row's
@@ -97,7 +104,7 @@ template <> struct RawRow<16> {
     }
 };
 
-template <int KIND, int BITS>
+template <int KIND, int BITS, bool PIVOT>
 __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, DecodeIO io)
 {
     __shared__ __align__(16) float red[kRawThreads / 32][2][kD];  // column partials per warp
@@ -108,13 +115,15 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
 
     const int tile = blockIdx.x;
     const int ni = tile / p.H, h = tile - ni * p.H;
+    if (PIVOT && p.t.row_bits[h * kD] != 16) return;  // a quantized head: the fused kernel's
     const int req = io.req_idx[ni], slot = io.slot_idx[ni];
     const int tid = threadIdx.x;
     if (req < 0 || req >= p.R || slot < 0 || slot >= p.S) {  // uniform over the CTA
         if (tid == 0) atomicOr(p.err, kErrIndex);
         return;
     }
-    uint8_t *page = p.pages + (static_cast<size_t>(req) * p.S + slot) * p.slot_bytes + p.t.head_off[h];
+    uint8_t *page = p.pages + (static_cast<size_t>(req) * p.S + slot) * p.slot_bytes + p.t.head_off[h] +
+                    (PIVOT ? p.scale_bytes * kD : 0);
     const size_t vec = static_cast<size_t>(tile) * kD;
     const int warp = tid >> 5, lane = tid & 31;
     const int rgl = lane >> 4, cg = lane & 15;
@@ -132,9 +141,10 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
         const int r = tid - kD;
         const float g = KIND == STQ_GDN ? io.gate[tile] : io.gate[vec + r];
         const float k = io.k[vec + r], q = io.q[vec + r];
-        gk[r] = g * k;
-        gq[r] = g * q;
-        ks[r] = k;
+        const float rr = PIVOT ? p.t.r[h * kD + r] : 1.0f;
+        gk[r] = PIVOT ? (g * k) * rr : g * k;
+        gq[r] = PIVOT ? (g * q) * rr : g * q;
+        ks[r] = PIVOT ? __fdiv_rn(k, rr) : k;
         float a = k * q;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
@@ -180,10 +190,11 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
             yz += red[w][1][j];
         }
         const float kq = (kqp[0] + kqp[1]) + (kqp[2] + kqp[3]);
-        const float u = io.beta[tile] * (io.v[vec + j] - vz);
-        const float yj = fmaf(kq, u, yz);
+        const float cj = PIVOT ? p.t.c[h * kD + j] : 1.0f;
+        const float u = io.beta[tile] * (io.v[vec + j] - (PIVOT ? cj * vz : vz));
+        const float yj = fmaf(kq, u, PIVOT ? cj * yz : yz);
         io.y[vec + j] = yj;
-        us[j] = u;
+        us[j] = PIVOT ? __fdiv_rn(u, cj) : u;
         if (!isfinite(u) || !isfinite(yj)) atomicOr(&bad, 1u);
     }
     __syncthreads();
@@ -215,15 +226,20 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
     if (tid == 0 && bad) atomicOr(p.err, kErrNonFinite);
 }
 
-template <int KIND, int BITS>
+template <int KIND, int BITS, bool PIVOT = false>
 cudaError_t launch_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
-    decode_raw_kernel<KIND, BITS><<<io.n * p.H, kRawThreads, 0, stream>>>(p, io);
+    decode_raw_kernel<KIND, BITS, PIVOT><<<io.n * p.H, kRawThreads, 0, stream>>>(p, io);
     count_launch();
     return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_decode_pivot_heads(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
+{
+    return launch_raw<STQ_GDN, 16, true>(p, io, stream);
+}
 
 cudaError_t launch_decode_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {

@@ -13,6 +13,7 @@ namespace stq {
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kScaleBytes = 4 * kD; // fp32 scales at the start of a page
 constexpr int kPageAlign = 128;    // pages are padded to this many bytes
+constexpr int kMaxStagedPage = kScaleBytes + 16 * 8 * kD;  // largest page the fused kernel stages (8 bits per row)
 constexpr size_t kStaticScratchFloats = size_t(1) << 20;  // built-in u~ buffer: 4 MiB, 8192 tiles
 
 // device error word bits
@@ -46,6 +47,7 @@ struct PoolView {
     int kind;
     int scale_bytes;     // bytes per row scale: 4 (fp32) or 2 (binary16); 0 in a raw pool
     int raw_bits;        // 16 or 32 in a raw pool (every unit), else 0
+    int pivots;          // nonzero if 16-bit (FP16 pivot) units sit among quantized ones
     Tables t;
     uint32_t *err;
 };
@@ -61,6 +63,8 @@ struct DecodeIO {
 
 cudaError_t launch_decode(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+// GDN FP16 pivot heads of a quantized pool (pages larger than kMaxStagedPage), one CTA per tile
+cudaError_t launch_decode_pivot_heads(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_readout(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_writeback(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,

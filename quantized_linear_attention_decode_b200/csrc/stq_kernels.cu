@@ -31,7 +31,8 @@ __device__ __forceinline__ uint8_t *tile_page(const PoolView &p, int req, int sl
 }
 
 // fp32 state -> packed page: mu = fl32(S / (r c)) (fp64 quotient), s = fl32(max|mu| / q_b),
-// z = clip(rint(fl32(mu / s)), -q_b, q_b).  One warp per row.
+// z = clip(rint(fl32(mu / s)), -q_b, q_b).  A 16-bit row is an FP16 pivot: its scale
+// slot holds 1 and it stores mu rounded once to binary16.  One warp per row.
 __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t *req_idx,
                                                        const int32_t *slot_idx, const float *state)
 {
@@ -64,6 +65,20 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        if (b == 16) {
+            const __half2 h01 = __floats2half2_rn(mu[0], mu[1]), h23 = __floats2half2_rn(mu[2], mu[3]);
+            uint2 w;
+            w.x = *reinterpret_cast<const uint32_t *>(&h01);
+            w.y = *reinterpret_cast<const uint32_t *>(&h23);
+            *reinterpret_cast<uint2 *>(page + p.t.row_off[h * kD + i] + lane * 8) = w;
+            const float2 f01 = __half22float2(h01), f23 = __half22float2(h23);
+            bad |= !(isfinite(f01.x) && isfinite(f01.y) && isfinite(f23.x) && isfinite(f23.y));
+            if (lane == 0) {
+                if (p.scale_bytes == 2) reinterpret_cast<__half *>(page)[i] = __float2half_rn(1.0f);
+                else reinterpret_cast<float *>(page)[i] = 1.0f;
+            }
+            continue;
+        }
         float s = __fdiv_rn(a, static_cast<float>(qb));
         __half s16 = __float2half_rn(s);
         if (p.scale_bytes == 2) s = __half2float(s16);  // the scale as stored
@@ -100,7 +115,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrNonFinite);
 }
 
-// packed page -> fp32 reconstruction fl32(((s r) c) z) computed in fp64.  One warp per row.
+// packed page -> fp32 reconstruction fl32(((s r) c) z) computed in fp64 (z: the binary16
+// value of a pivot row).  One warp per row.
 __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32_t *req_idx,
                                                          const int32_t *slot_idx, float *state)
 {
@@ -122,8 +138,16 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
                                             : reinterpret_cast<const float *>(page)[i];
         const double sr = static_cast<double>(sc) * static_cast<double>(p.t.r[h * kD + i]);
         const uint8_t *row = page + p.t.row_off[h * kD + i];
-        int zz[4];
-        if (b == 8) {
+        double zz[4];
+        if (b == 16) {
+            const uint2 w = *reinterpret_cast<const uint2 *>(row + lane * 8);
+            const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&w.x));
+            const float2 c2 = __half22float2(*reinterpret_cast<const __half2 *>(&w.y));
+            zz[0] = a.x;
+            zz[1] = a.y;
+            zz[2] = c2.x;
+            zz[3] = c2.y;
+        } else if (b == 8) {
             const uint32_t w = *reinterpret_cast<const uint32_t *>(row + lane * 4);
 #pragma unroll
             for (int t = 0; t < 4; ++t) zz[t] = static_cast<int>(w << (24 - 8 * t)) >> 24;
@@ -137,10 +161,10 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
             for (int t = 0; t < 4; ++t) zz[t] = static_cast<int>(w << (26 - 6 * t)) >> 26;
         }
         float4 o;
-        o.x = static_cast<float>(sr * static_cast<double>(cj[0]) * static_cast<double>(zz[0]));
-        o.y = static_cast<float>(sr * static_cast<double>(cj[1]) * static_cast<double>(zz[1]));
-        o.z = static_cast<float>(sr * static_cast<double>(cj[2]) * static_cast<double>(zz[2]));
-        o.w = static_cast<float>(sr * static_cast<double>(cj[3]) * static_cast<double>(zz[3]));
+        o.x = static_cast<float>(sr * static_cast<double>(cj[0]) * zz[0]);
+        o.y = static_cast<float>(sr * static_cast<double>(cj[1]) * zz[1]);
+        o.z = static_cast<float>(sr * static_cast<double>(cj[2]) * zz[2]);
+        o.w = static_cast<float>(sr * static_cast<double>(cj[3]) * zz[3]);
         *reinterpret_cast<float4 *>(S + i * kD + lane * 4) = o;
     }
 }

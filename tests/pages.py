@@ -12,10 +12,13 @@ import numpy as np
 D = 128
 
 
+PIVOT = 4  # format flag: 16-bit rows are FP16 pivots among quantized rows
+
+
 def _scale_bytes(row_bits, fmt) -> int:
-    if int(np.asarray(row_bits).reshape(-1)[0]) in (16, 32):
+    if not (fmt & PIVOT) and int(np.asarray(row_bits).reshape(-1)[0]) in (16, 32):
         return 0  # raw page
-    return 2 if fmt == 1 else 4
+    return 2 if fmt & 1 else 4
 
 
 def page_bytes(row_bits, fmt: int = 0) -> int:
@@ -43,7 +46,7 @@ def raw_values(page: np.ndarray, row_bits) -> np.ndarray:
 def decode_page(page: np.ndarray, row_bits, fmt: int = 0) -> tuple[np.ndarray, np.ndarray]:
     """(scales float32 [128], codes int32 [128, 128]) of one page."""
     page = np.asarray(page, np.uint8)
-    if fmt == 1:
+    if fmt & 1:
         scales = page[: 2 * D].view(np.float16).astype(np.float32)
     else:
         scales = page[: 4 * D].view(np.float32).copy()
@@ -59,6 +62,16 @@ def decode_page(page: np.ndarray, row_bits, fmt: int = 0) -> tuple[np.ndarray, n
         u = (bits << np.arange(b)).sum(axis=2)
         codes[rows] = np.where(u >= (1 << (b - 1)), u - (1 << b), u)
     return scales, codes
+
+
+def pivot_values(page: np.ndarray, row_bits, fmt: int = PIVOT) -> np.ndarray:
+    """[128, 128] binary16 values of the pivot (16-bit) rows as float64; NaN elsewhere."""
+    page = np.asarray(page, np.uint8)
+    out = np.full((D, D), np.nan)
+    offs = row_offsets(row_bits, fmt)
+    for i in np.nonzero(np.asarray(row_bits) == 16)[0]:
+        out[i] = page[offs[i]: offs[i] + 2 * D].view(np.float16).astype(np.float64)
+    return out
 
 
 def split_slot(slot: np.ndarray, pool_row_bits, fmt: int = 0) -> list[np.ndarray]:
@@ -113,10 +126,14 @@ class Compare:
     def page(self, page_gpu, page_ref, quot, row_bits, where="", fmt=0):
         sg, zg = decode_page(page_gpu, row_bits, fmt)
         sr, zr = decode_page(page_ref, row_bits, fmt)
-        self.codes += zg.size
+        piv = np.asarray(row_bits) == 16
+        if piv.any():
+            self._pivots(page_gpu, page_ref, quot, row_bits, piv, where, fmt)
+            assert np.all(sg[piv] == 1) and np.all(sr[piv] == 1), f"pivot scale slot not 1 {where}"
+        self.codes += int((~piv).sum()) * D
         qref = np.asarray(quot, np.float64).copy()
         zref = zr.copy()
-        if fmt == 1:
+        if fmt & 1:
             # binary16 scales: a row whose s = a / q_b lies next to a rounding midpoint of
             # binary16 may round to the other neighbour on the GPU (its a differs by an ulp
             # or two); then its codes follow the GPU's scale
@@ -144,13 +161,29 @@ class Compare:
                 f"cols {jj[bad][:5]}, gpu {zg[ii, jj][bad][:5]}, ref {zref[ii, jj][bad][:5]}, quot {x[bad][:5]}")
             for a, b in zip(ii, jj):
                 self.ties.append((where, int(a), int(b), float(qref[a, b]), int(zg[a, b]), int(zref[a, b])))
-        if fmt == 1:
+        if fmt & 1:
             return  # every scale is equal or an accepted flip
         den = np.maximum(np.abs(sr.astype(np.float64)), 1e-38)
         rel = np.abs(sg.astype(np.float64) - sr) / den
         rel[(sr == 0) & (sg == 0)] = 0.0
         self.worst_s = max(self.worst_s, float(rel.max()))
         assert rel.max() <= self.rtol, f"scale rel err {rel.max():.3g} {where}"
+
+    def _pivots(self, page_gpu, page_ref, quot, row_bits, piv, where, fmt):
+        """FP16 pivot rows: binary16 values of mu = X / (r c), equal except where the
+        GPU's value rounds a value within raw_tie_rel x max|mu| (over the unit's pivot
+        rows) of the oracle's fl32(mu), passed in quot."""
+        xg, xr = pivot_values(page_gpu, row_bits, fmt)[piv], pivot_values(page_ref, row_bits, fmt)[piv]
+        self.values += xg.size
+        diff = xg != xr
+        if diff.any():
+            M = np.asarray(quot, np.float64)[piv]
+            x = M[diff]
+            half_ulp = np.abs(np.spacing(xg[diff].astype(np.float16)).astype(np.float64)) / 2
+            near = np.abs(xg[diff] - x) <= self.raw_tie_rel * np.abs(M).max() + half_ulp
+            assert near.all(), (f"{int((~near).sum())} pivot mismatches beyond the fp32 error window {where}: "
+                                f"gpu {xg[diff][~near][:5]} ref {xr[diff][~near][:5]} mu {x[~near][:5]}")
+            self.raw_ties += int(diff.sum())
 
     def raw(self, page_gpu, page_ref, quot, row_bits, where=""):
         """A raw page: fp32 values within rtol of the unit's largest; binary16

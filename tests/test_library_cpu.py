@@ -91,9 +91,21 @@ def test_desc_bytes_formats():
     assert s32 == 2 * s16
 
 
+def test_desc_bytes_pivot_pool():
+    """16-bit units among quantized ones are FP16 pivots: every page keeps its scale
+    section, a pivot head holds 128 rows of 256 B."""
+    for flags, sb in ((0, 512), (stq.STQ_SCALE_F16, 256)):
+        bits = np.array([16, 6, 8, 16], np.uint8)
+        _, slot = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits, flags=flags)
+        assert slot == sum(sb + 2048 * int(b) for b in bits)
+        kb = np.tile(np.array([16] + [6] * 127, np.uint8), 2)
+        _, slot = stq.stq_desc_bytes(stq.STQ_KDA, 1, 1, 2, kb, flags=flags)
+        assert slot == 2 * ((sb + 256 + 127 * 96 + 127) // 128 * 128)
+
+
 @pytest.mark.parametrize("ub, flags, status", [
-    ([16, 16, 8, 16], 0, "STQ_ERR_UNSUPPORTED"),  # raw and quantized units mixed
     ([32, 16, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),  # two raw widths
+    ([32, 8, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),   # fp32 units among quantized ones
     ([16, 16, 16, 16], 1, "STQ_ERR_ARG"),          # a raw pool has no scales
     ([6, 6, 6, 6], 2, "STQ_ERR_ARG"),              # unknown flag
     ([6, 12, 6, 6], 0, "STQ_ERR_ARG"),
