@@ -54,6 +54,9 @@ def lib():
         L.orc_dequantize_unit_fmt.argtypes = [C.c_int, C.c_int, P, P, P, C.c_int, P, P]
         L.orc_step_unit_fmt.argtypes = [C.c_int, C.c_int, P, P, P, C.c_int, P, P, P, P, P,
                                         C.c_float, P, P, P]
+        L.orc_quantize_unit_w.argtypes = [C.c_int, C.c_int, P, P, P, P, C.c_int, P, P, P]
+        L.orc_step_unit_w.argtypes = [C.c_int, C.c_int, P, P, P, P, C.c_int, P, P, P, P, P,
+                                      C.c_float, P, P, P]
         L.orc_get_code.restype = C.c_int32
         L.orc_get_code.argtypes = [P, C.c_int, C.c_int]
         L.orc_put_code.restype = None
@@ -89,7 +92,7 @@ def _f64(a):
 # 16-bit rows are FP16 pivots among quantized rows (scale slot 1, binary16
 # mu = X / (r c)).  Without the flag, units whose rows are all 16 or all 32
 # bits wide are raw (binary16 / binary32 values, no scales).
-FMT_F32, FMT_F16, FMT_PIVOT = 0, 1, 4
+FMT_F32, FMT_F16, FMT_PIVOT, FMT_FITC = 0, 1, 4, 8
 
 
 def is_raw(bits, fmt: int = FMT_F32) -> bool:
@@ -108,7 +111,8 @@ def row_offsets(bits, dv: int | None = None, fmt: int = FMT_F32) -> np.ndarray:
     dv = len(bits) if dv is None else dv
     sizes = dv * bits // 8
     sb = 0 if is_raw(bits, fmt) else (2 if fmt & FMT_F16 else 4)
-    return sb * len(bits) + np.concatenate([[0], np.cumsum(sizes)[:-1]])
+    cf = 4 * dv if fmt & FMT_FITC else 0  # the page's own column factors
+    return sb * len(bits) + cf + np.concatenate([[0], np.cumsum(sizes)[:-1]])
 
 
 def half_to_double(h: int) -> float:
@@ -131,15 +135,17 @@ def put_code(row: np.ndarray, b: int, j: int, z: int) -> None:
     lib().orc_put_code(_p(row), b, j, int(z))
 
 
-def quantize_unit(bits, r, c, S, *, with_quot: bool = False, fmt: int = FMT_F32):
+def quantize_unit(bits, r, c, S, *, with_quot: bool = False, fmt: int = FMT_F32, w=None):
     """fp32 state [dk, dv] -> packed page (uint8).  Optionally the fp32
-    quotients mu / s the codes were rounded from."""
+    quotients mu / s the codes were rounded from.  w: row weights of the
+    column fit (FMT_FITC; None for 1)."""
     bits, r, c, S = _u8(bits), _f32(r), _f32(c), _f32(S)
+    w = None if w is None else _f32(w)
     dk, dv = S.shape
     page = np.zeros(page_bytes(bits, dv, fmt), np.uint8)
     quot = np.zeros((dk, dv), np.float32) if with_quot else None
-    st = lib().orc_quantize_unit_fmt(dk, dv, _p(bits), _p(r), _p(c), int(fmt), _p(S), _p(page),
-                                     _p(quot))
+    st = lib().orc_quantize_unit_w(dk, dv, _p(bits), _p(r), _p(c), _p(w), int(fmt), _p(S), _p(page),
+                                   _p(quot))
     if st == BADARG:
         raise ValueError("bad bit widths")
     return (page, quot, st) if with_quot else page
@@ -156,13 +162,14 @@ def dequantize_unit(bits, r, c, page, dv: int | None = None, fmt: int = FMT_F32)
     return S
 
 
-def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None, fmt: int = FMT_F32):
+def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None, fmt: int = FMT_F32, w=None):
     """One quantized decode step of one unit.
 
     Returns (page_out uint8, y float64 [dv], quot float32 [dk, dv], status).
     For a raw unit quot holds fl32(X), the value before its rounding on store."""
     bits, r, c, page_in = _u8(bits), _f32(r), _f32(c), _u8(page_in)
     q, k, v, g = _f32(q), _f32(k), _f32(v), _f32(g)
+    w = None if w is None else _f32(w)
     dk = len(bits)
     dv = len(v) if dv is None else dv
     if g.size == 1:
@@ -170,9 +177,9 @@ def step_unit(bits, r, c, page_in, q, k, v, beta, g, dv: int | None = None, fmt:
     page_out = np.zeros(page_bytes(bits, dv, fmt), np.uint8)
     y = np.zeros(dv, np.float64)
     quot = np.zeros((dk, dv), np.float32)
-    st = lib().orc_step_unit_fmt(dk, dv, _p(bits), _p(r), _p(c), int(fmt), _p(page_in),
-                                 _p(page_out), _p(q), _p(k), _p(v), float(beta), _p(g), _p(y),
-                                 _p(quot))
+    st = lib().orc_step_unit_w(dk, dv, _p(bits), _p(r), _p(c), _p(w), int(fmt), _p(page_in),
+                               _p(page_out), _p(q), _p(k), _p(v), float(beta), _p(g), _p(y),
+                               _p(quot))
     if st == BADARG:
         raise ValueError("bad bit widths")
     return page_out, y, quot, st

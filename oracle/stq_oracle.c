@@ -47,6 +47,19 @@
  *     mu_ij = fl32(X_ij / (r_i c_j)) rounded once to binary16 in place of
  *     the codes; it reconstructs as s_i r_i c_j mu_ij like a quantized row
  *     (with r = c = 1, the state value itself);
+ *   - online column fit ([core]: c_j minimises sum_{i,j} w_i^2 (X_ij -
+ *     r_i c_j z_ij)^2; [steps] steps 4-5, closed form c_j = sum_i w_i^2
+ *     v_ij X_ij / sum_i w_i^2 v_ij^2 with the page's garbled v_ij read as the
+ *     row's reconstruction without c, r_i s_i z_ij; format flag 8): the page
+ *     carries its own dv fp32 column factors after the scales.  Each
+ *     quantisation takes the codes with the page's current factors (one pass,
+ *     no iteration between codes and factors), then refits every column over
+ *     the unit's rows with the frozen row weights w_i and stores the new
+ *     factors; a column whose codes are all zero keeps its factor.  With one
+ *     absmax scale per row, r_i cancels from codes and reconstruction alike,
+ *     so the row factor's online formula r_i = m_i^(1/2) w_i^(-1/2) changes
+ *     nothing here and is not evaluated.  Pivot rows are not combined with
+ *     the fit;
  *   - the continuous part (reconstruction, decay, retrieval, write,
  *     readout) is computed in fp64; the quantisation decision is taken in
  *     fp32 on the fp32-rounded value mu_ij = fl32(X_ij / (r_i c_j)), with
@@ -79,11 +92,17 @@ static int q_of_bits(int b) { return (1 << (b - 1)) - 1; }
 
 static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8u; }
 
-/* format flags: bit 0 binary16 scales, bit 2 FP16 pivot rows among quantized ones */
+/* format flags: bit 0 binary16 scales, bit 2 FP16 pivot rows among quantized ones,
+ * bit 3 per-page column factors fitted at every quantisation */
 #define ORC_FMT_F16 1
 #define ORC_FMT_PIVOT 4
+#define ORC_FMT_FITC 8
 
-static int fmt_ok(int fmt) { return fmt >= 0 && (fmt & ~(ORC_FMT_F16 | ORC_FMT_PIVOT)) == 0; }
+static int fmt_ok(int fmt)
+{
+    if (fmt < 0 || (fmt & ~(ORC_FMT_F16 | ORC_FMT_PIVOT | ORC_FMT_FITC)) != 0) return 0;
+    return !((fmt & ORC_FMT_PIVOT) && (fmt & ORC_FMT_FITC));
+}
 
 /* 16 or 32 for a raw unit (its first row decides; bits_ok checks the rest), else 0 */
 static int raw_width(int dk, const uint8_t *bits, int fmt)
@@ -117,9 +136,12 @@ static size_t scale_bytes(int dk, const uint8_t *bits, int fmt)
     return (fmt & ORC_FMT_F16) ? 2u : 4u;
 }
 
+/* bytes of the column-factor section (fp32, after the scales) */
+static size_t colf_bytes(int dv, int fmt) { return (fmt & ORC_FMT_FITC) ? 4u * (size_t)dv : 0u; }
+
 size_t orc_page_bytes_fmt(int dk, int dv, const uint8_t *bits, int fmt)
 {
-    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk;
+    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk + colf_bytes(dv, fmt);
     for (int i = 0; i < dk; ++i) n += row_bytes(dv, bits[i]);
     return (n + 127u) / 128u * 128u;
 }
@@ -128,7 +150,7 @@ size_t orc_page_bytes(int dk, int dv, const uint8_t *bits) { return orc_page_byt
 
 static size_t row_offset(int dk, int dv, const uint8_t *bits, int fmt, int i)
 {
-    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk;
+    size_t n = scale_bytes(dk, bits, fmt) * (size_t)dk + colf_bytes(dv, fmt);
     for (int t = 0; t < i; ++t) n += row_bytes(dv, bits[t]);
     return n;
 }
@@ -243,6 +265,20 @@ static double put_raw(uint8_t *row, int b, int j, double x)
     return (double)f;
 }
 
+/* column factor j of a unit: the page's own under ORC_FMT_FITC, else the frozen table */
+static float col_factor(const uint8_t *page, int dk, const uint8_t *bits, int fmt, const float *c, int j)
+{
+    if (!(fmt & ORC_FMT_FITC)) return c[j];
+    float f;
+    memcpy(&f, page + scale_bytes(dk, bits, fmt) * (size_t)dk + 4 * (size_t)j, 4);
+    return f;
+}
+
+static void put_col_factor(uint8_t *page, int dk, const uint8_t *bits, int fmt, int j, float f)
+{
+    memcpy(page + scale_bytes(dk, bits, fmt) * (size_t)dk + 4 * (size_t)j, &f, 4);
+}
+
 /* exported for the pack/unpack pins */
 int32_t orc_get_code(const uint8_t *row, int b, int j) { return get_code(row, b, j); }
 void orc_put_code(uint8_t *row, int b, int j, int32_t z) { put_code(row, b, j, z); }
@@ -262,19 +298,48 @@ static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, con
         double s = (double)get_scale(page, fmt, i);
         for (int j = 0; j < dv; ++j) {
             double z = bits[i] == 16 ? get_raw(row, 16, j) : (double)get_code(row, bits[i], j);
-            S[(size_t)i * dv + j] = s * (double)r[i] * (double)c[j] * z;
+            double cj = (double)col_factor(page, dk, bits, fmt, c, j);
+            S[(size_t)i * dv + j] = s * (double)r[i] * cj * z;
         }
     }
+}
+
+/*
+ * [core], [steps] steps 4-5: the weighted least-squares column factors of the
+ * codes just written, c_j = sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2 with
+ * v_ij = s_i r_i z_ij, in fp64, stored as fp32 (a column whose codes are all
+ * zero keeps c_old).  Returns ORC_NONFINITE if a factor is not finite.
+ */
+static int fit_columns(int dk, int dv, const uint8_t *bits, const float *r, const float *c_old,
+                       const float *w, int fmt, const double *X, uint8_t *page)
+{
+    int status = ORC_OK;
+    for (int j = 0; j < dv; ++j) {
+        double num = 0.0, den = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            const uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
+            double v = (double)get_scale(page, fmt, i) * (double)r[i] * (double)get_code(row, bits[i], j);
+            double wi = w ? (double)w[i] : 1.0;
+            num += wi * wi * v * X[(size_t)i * dv + j];
+            den += wi * wi * v * v;
+        }
+        float cj = den > 0.0 ? (float)(num / den) : c_old[j];
+        if (!isfinite(cj)) status = ORC_NONFINITE;
+        put_col_factor(page, dk, bits, fmt, j, cj);
+    }
+    return status;
 }
 
 /*
  * [bg-quant], [bg-smooth], [core], [steps] steps 4-6: quantise X row by row
  * and write scales and codes into page.  quot (optional) receives the fp32
  * quotient mu_ij / s_i that round() is applied to (for near-tie analysis).
- * Returns ORC_NONFINITE if a row maximum is not finite.
+ * c holds the column factors the codes are taken with (the unit's current
+ * ones); under ORC_FMT_FITC the page then receives refitted factors (row
+ * weights w, NULL for 1).  Returns ORC_NONFINITE if a row maximum is not finite.
  */
 static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                      int fmt, const double *X, uint8_t *page, float *quot)
+                      const float *w, int fmt, const double *X, uint8_t *page, float *quot)
 {
     int status = ORC_OK;
     int raw = raw_width(dk, bits, fmt);
@@ -333,21 +398,30 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
         }
     }
     free(mu);
+    if ((fmt & ORC_FMT_FITC) && fit_columns(dk, dv, bits, r, c, w, fmt, X, page) != ORC_OK) status = ORC_NONFINITE;
     return status;
 }
 
-/* fp32 state -> packed page (the quantizer applied to a given state) */
-int orc_quantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                          int fmt, const float *S, uint8_t *page, float *quot)
+/* fp32 state -> packed page (the quantizer applied to a given state; under
+ * ORC_FMT_FITC the codes are taken with the table's factors c and the page
+ * receives the refitted ones) */
+int orc_quantize_unit_w(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                        const float *w, int fmt, const float *S, uint8_t *page, float *quot)
 {
     if (!bits_ok(dk, dv, bits, fmt)) return ORC_BADARG;
     size_t nb = orc_page_bytes_fmt(dk, dv, bits, fmt);
     memset(page, 0, nb);
     double *X = (double *)malloc(sizeof(double) * (size_t)dk * dv);
     for (size_t e = 0; e < (size_t)dk * dv; ++e) X[e] = (double)S[e];
-    int st = requantize(dk, dv, bits, r, c, fmt, X, page, quot);
+    int st = requantize(dk, dv, bits, r, c, w, fmt, X, page, quot);
     free(X);
     return st;
+}
+
+int orc_quantize_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                          int fmt, const float *S, uint8_t *page, float *quot)
+{
+    return orc_quantize_unit_w(dk, dv, bits, r, c, NULL, fmt, S, page, quot);
 }
 
 int orc_quantize_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
@@ -386,10 +460,10 @@ int orc_dequantize_unit(int dk, int dv, const uint8_t *bits, const float *r, con
  * y is returned in fp64; quot (optional, dk*dv floats) receives the fp32
  * quotients the new codes were rounded from.
  */
-int orc_step_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
-                      int fmt, const uint8_t *page_in, uint8_t *page_out,
-                      const float *q, const float *k, const float *v, float beta, const float *g,
-                      double *y, float *quot)
+int orc_step_unit_w(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                    const float *w, int fmt, const uint8_t *page_in, uint8_t *page_out,
+                    const float *q, const float *k, const float *v, float beta, const float *g,
+                    double *y, float *quot)
 {
     if (!bits_ok(dk, dv, bits, fmt)) return ORC_BADARG;
     size_t nel = (size_t)dk * dv;
@@ -412,14 +486,26 @@ int orc_step_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const
         for (int i = 0; i < dk; ++i) acc += (double)q[i] * P[(size_t)i * dv + j];
         y[j] = acc;
     }
+    /* the codes are taken with the unit's current column factors */
+    float *c_now = (float *)malloc(sizeof(float) * (size_t)dv);
+    for (int j = 0; j < dv; ++j) c_now[j] = col_factor(page_in, dk, bits, fmt, c, j);
     memset(page_out, 0, orc_page_bytes_fmt(dk, dv, bits, fmt));
-    int st = requantize(dk, dv, bits, r, c, fmt, P, page_out, quot);
+    int st = requantize(dk, dv, bits, r, c_now, w, fmt, P, page_out, quot);
+    free(c_now);
     for (int j = 0; j < dv; ++j)
         if (!isfinite(y[j])) st = ORC_NONFINITE;
     free(P);
     free(vo);
     free(u);
     return st;
+}
+
+int orc_step_unit_fmt(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
+                      int fmt, const uint8_t *page_in, uint8_t *page_out,
+                      const float *q, const float *k, const float *v, float beta, const float *g,
+                      double *y, float *quot)
+{
+    return orc_step_unit_w(dk, dv, bits, r, c, NULL, fmt, page_in, page_out, q, k, v, beta, g, y, quot);
 }
 
 int orc_step_unit(int dk, int dv, const uint8_t *bits, const float *r, const float *c,
