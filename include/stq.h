@@ -76,6 +76,14 @@ typedef struct stq_pool stq_pool;
  * units mixed with others return STQ_ERR_UNSUPPORTED.
  */
 #define STQ_SCALE_F16 1u /* flags: per-row scales stored as IEEE binary16 ("method steps", step 6) */
+/* flags: every page carries its own column factors c_j, refitted at each
+ * quantisation ("core method" dual-axis fit; "method steps", steps 4-5):
+ * the codes are taken with the page's current factors, then
+ *   c_j <- sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2,  v_ij = s_i r_i z_ij,
+ * over the head's rows with the frozen row weights w_i (row_weight); a column
+ * whose codes are all zero keeps its factor.  col_factor gives the factors
+ * the first quantisation starts from.  Not with pivot or raw units. */
+#define STQ_FIT_COLUMNS 2u
 
 typedef struct {
     int32_t kind;         /* stq_kind */
@@ -87,7 +95,11 @@ typedef struct {
     const uint8_t *unit_bits;  /* host; GDN: [H] one width per head; KDA: [H * d_k] one per key row */
     const float *row_factor;   /* host; [H * d_k] r_i, finite and > 0; NULL means all 1 */
     const float *col_factor;   /* host; [H * d_v] c_j, finite and > 0; NULL means all 1 */
-    uint32_t flags;            /* 0 (fp32 scales) or STQ_SCALE_F16; must be 0 for a raw pool */
+    uint32_t flags;            /* STQ_SCALE_F16 | STQ_FIT_COLUMNS, or 0; must be 0 for a raw pool */
+    const float *row_weight;   /* host; [H * d_k] w_i > 0, finite: row influence weights of the
+                                  column fit ("core method": w_i, the gamma = 0.25 power of the
+                                  calibrated influence omega_i, geometric-mean normalised);
+                                  NULL means all 1; read only with STQ_FIT_COLUMNS */
 } stq_pool_desc;
 
 /*
@@ -97,6 +109,7 @@ typedef struct {
  *                    rounded from mu / s16 so that s16 z reconstructs them,
  *                    and a scale beyond the binary16 range is reported as
  *                    STQ_ERR_NONFINITE)
+ *   with STQ_FIT_COLUMNS: then 128 fp32 column factors c_j of this page
  *   then rows i = 0..127 in order, row i holding 128 codes of b_i bits
  *   (16 * b_i bytes); code j occupies bits [j b_i, (j+1) b_i) of the row's
  *   little-endian bit string, as a b_i-bit two's complement integer in
@@ -104,7 +117,8 @@ typedef struct {
  *   zero padding up to a multiple of 128 bytes.
  * The pages of heads 0..H-1 follow each other inside a slot; slots are
  * ordered [request][slot].  The state the page stands for is
- *   S^_ij = s_i * r_i * c_j * z_ij          ("core method": X^ = r c z).
+ *   S^_ij = s_i * r_i * c_j * z_ij          ("core method": X^ = r c z),
+ * with c_j the pool's column factors, or the page's own with STQ_FIT_COLUMNS.
  * A raw page (units of 16 or 32 bits) is the row-major 128 x 128 state in
  * binary16 or fp32 (32 KiB or 64 KiB), with no scales; r and c do not apply,
  * and every step rounds X once (to nearest even) into it.

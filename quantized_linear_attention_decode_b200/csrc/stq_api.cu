@@ -18,6 +18,7 @@ struct stq_pool {
     int scale_bytes = 4, raw_bits = 0;
     bool pivots = false;       // FP16 pivot units among quantized ones
     bool pivot_heads = false;  // GDN pivot heads (their own kernel)
+    bool fit = false;          // per-page column factors refitted at every quantisation
     int device = 0;
     size_t slot_bytes = 0, packed_bytes = 0;
     uint8_t *d_pages = nullptr;
@@ -65,10 +66,10 @@ struct HeadLayout {
     uint16_t row_off[stq::kD];
 };
 
-HeadLayout head_layout(const uint8_t *row_bits, int scale_bytes)
+HeadLayout head_layout(const uint8_t *row_bits, int scale_bytes, bool fit)
 {
     HeadLayout L{};
-    uint32_t off = (uint32_t)scale_bytes * stq::kD;
+    uint32_t off = (uint32_t)scale_bytes * stq::kD + (fit ? (uint32_t)stq::kFitBytes : 0u);
     for (int i = 0; i < stq::kD; ++i) {
         L.row_off[i] = (uint16_t)off;
         off += 16u * row_bits[i];
@@ -108,7 +109,7 @@ stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
     if (d->unit_bits == nullptr) return fail(STQ_ERR_ARG, "unit_bits is NULL");
     const int H = d->num_heads;
     const size_t nunits = d->kind == STQ_GDN ? (size_t)H : (size_t)H * stq::kD;
-    if (d->flags & ~STQ_SCALE_F16) return fail(STQ_ERR_ARG, "flags 0x%x", d->flags);
+    if (d->flags & ~(STQ_SCALE_F16 | STQ_FIT_COLUMNS)) return fail(STQ_ERR_ARG, "flags 0x%x", d->flags);
     for (size_t u = 0; u < nunits; ++u) {
         int b = d->unit_bits[u];
         if (b != 4 && b != 6 && b != 8 && b != 16 && b != 32)
@@ -120,6 +121,14 @@ stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
             if (d->unit_bits[u] == 32)
                 return fail(STQ_ERR_UNSUPPORTED, "unit_bits[%zu] = 32: fp32 units must make up the whole pool", u);
     if (raw && d->flags != 0) return fail(STQ_ERR_ARG, "a raw pool has no scales (flags must be 0)");
+    if (d->flags & STQ_FIT_COLUMNS)
+        for (size_t u = 0; u < nunits; ++u)
+            if (d->unit_bits[u] == 16)
+                return fail(STQ_ERR_UNSUPPORTED, "STQ_FIT_COLUMNS with FP16 pivot units (unit_bits[%zu] = 16)", u);
+    if ((d->flags & STQ_FIT_COLUMNS) && d->row_weight)
+        for (size_t e = 0; e < (size_t)H * stq::kD; ++e)
+            if (!(std::isfinite(d->row_weight[e]) && d->row_weight[e] > 0.0f))
+                return fail(STQ_ERR_ARG, "row_weight[%zu] = %g (must be finite and > 0)", e, (double)d->row_weight[e]);
     for (int which = 0; which < 2; ++which) {
         const float *f = which ? d->col_factor : d->row_factor;
         if (f == nullptr) continue;
@@ -145,7 +154,7 @@ stq_status sizes_of(const stq_pool_desc *d, const std::vector<uint8_t> &row_bits
     size_t off = 0;
     const int sb = scale_bytes_of(d);
     for (int h = 0; h < d->num_heads; ++h) {
-        HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD], sb);
+        HeadLayout L = head_layout(&row_bits[(size_t)h * stq::kD], sb, (d->flags & STQ_FIT_COLUMNS) != 0);
         if (d->kind == STQ_KDA && sb != 0 && L.page_bytes > (uint32_t)stq::kMaxStagedPage)
             return fail(STQ_ERR_UNSUPPORTED, "KDA head %d: %u-byte page (FP16 pivot rows average above 8 bits "
                         "per row); at most %d bytes", h, L.page_bytes, stq::kMaxStagedPage);
@@ -173,6 +182,7 @@ stq::PoolView view(stq_pool *p)
     v.scale_bytes = p->scale_bytes;
     v.raw_bits = p->raw_bits;
     v.pivots = p->pivots ? 1 : 0;
+    v.fit = p->fit ? 1 : 0;
     v.t = p->t;
     v.err = p->d_err;
     return v;
@@ -319,6 +329,7 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->raw_bits = raw_width_of(desc);
     for (size_t u = 0; !p->raw_bits && u < rb.size(); ++u) p->pivots |= rb[u] == 16;
     p->pivot_heads = p->pivots && p->kind == STQ_GDN;
+    p->fit = (desc->flags & STQ_FIT_COLUMNS) != 0;
     st = sizes_of(desc, rb, &p->head_off, &p->page_bytes, &p->slot_bytes, &p->packed_bytes);
     if (st != STQ_OK) {
         delete p;
@@ -332,20 +343,22 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     const size_t n_blk = (size_t)H * stq::kHeadBlock;
     const size_t o_hoff = 0, o_pb = o_hoff + al(n_hoff), o_ro = o_pb + al(n_pb),
                  o_rb = o_ro + al(n_ro), o_r = o_rb + al(n_rb), o_c = o_r + al(n_f),
-                 o_blk = o_c + al(n_f), total = o_blk + al(n_blk);
+                 o_w = o_c + al(n_f), o_blk = o_w + al(n_f), total = o_blk + al(n_blk);
     std::vector<uint8_t> img(total, 0);
     std::memcpy(&img[o_hoff], p->head_off.data(), n_hoff);
     std::memcpy(&img[o_pb], p->page_bytes.data(), n_pb);
     for (int h = 0; h < H; ++h) {
-        HeadLayout L = head_layout(&rb[(size_t)h * kD], p->scale_bytes);
+        HeadLayout L = head_layout(&rb[(size_t)h * kD], p->scale_bytes, p->fit);
         std::memcpy(&img[o_ro + (size_t)h * kD * 2], L.row_off, kD * 2);
     }
     std::memcpy(&img[o_rb], rb.data(), n_rb);
     float *fr = reinterpret_cast<float *>(&img[o_r]);
     float *fc = reinterpret_cast<float *>(&img[o_c]);
+    float *fw = reinterpret_cast<float *>(&img[o_w]);  // w_i, the column fit's row weights (1 without)
     for (size_t e = 0; e < (size_t)H * kD; ++e) {
         fr[e] = desc->row_factor ? desc->row_factor[e] : 1.0f;
         fc[e] = desc->col_factor ? desc->col_factor[e] : 1.0f;
+        fw[e] = (desc->flags & STQ_FIT_COLUMNS) && desc->row_weight ? desc->row_weight[e] : 1.0f;
     }
     for (int h = 0; h < H; ++h) {
         uint8_t *blk = &img[o_blk + (size_t)h * stq::kHeadBlock];
@@ -389,6 +402,7 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->t.row_bits = base + o_rb;
     p->t.r = reinterpret_cast<const float *>(base + o_r);
     p->t.c = reinterpret_cast<const float *>(base + o_c);
+    p->t.w = reinterpret_cast<const float *>(base + o_w);
     p->t.block = base + o_blk;
     *out = p;
     return STQ_OK;

@@ -73,6 +73,7 @@ struct __align__(16) RowCoef {
     float mrq[kD];     // e_i / (r_i q_b(i)) (1 / (r_i q_b) for a dropped row): s'_i = |mrq_i| max_j |w_ij|
     uint16_t off[kD];  // byte offset of row i inside the page
     uint8_t bits[kD];
+    float fb[kD];      // column fit: (w_i r_i)^2
     uint32_t deg[4];   // bit i: row i's old content is dropped (e_i = 0)
     uint8_t *page;     // the tile's page in global memory
     float kqp[4];      // k.q, partial sums of rows [32 w, 32 w + 32)
@@ -84,14 +85,28 @@ struct __align__(128) Smem {
     RowCoef rc[2];
     float red[2048];   // column partial sums [8 warps][v, y][128]; then row-max partials
     float rowinv[kD];  // per-row quantisation multiplier (pass 2)
+    float red2[2048];  // column fit partial sums [8 warps][num, den][128], finished in the next tile
+    float rowA[kD], rowB[kD];  // column fit row coefficients of pass 2: A = fa s', B = fb s'^2
+    float fitc[kD];    // the column factors the tile's codes were taken with
     float ut[kD];      // u_j / c_j
     uint8_t *stage_page[kStages];
+    const float *stage_w[kStages];  // the tile's head row weights (column fit)
     uint32_t stage_valid[kStages];
     float beta[kStages], alpha[kStages];
     uint32_t raw[8][5];  // {req, slot, head offset, page bytes, head} of tile k in raw[k % 8]
     uint32_t flags;
     unsigned long long full[kStages];
+    uint8_t *fit_page[2];    // page of the tile whose fit is pending, by tile parity
+    uint32_t fit_pending[2];
 };
+// arrays read or written as 16-byte vectors start on 16-byte boundaries
+static_assert(offsetof(Smem, red) % 16 == 0 && offsetof(Smem, rowinv) % 16 == 0 && offsetof(Smem, red2) % 16 == 0 &&
+                  offsetof(Smem, ut) % 16 == 0 && offsetof(Smem, full) % 8 == 0 && offsetof(Smem, rc) % 16 == 0,
+              "shared-memory layout");
+static_assert(offsetof(Stage, q) % 16 == 0 && offsetof(Stage, k) % 16 == 0 && offsetof(Stage, v) % 16 == 0 &&
+                  offsetof(Stage, g) % 16 == 0 && offsetof(Stage, r) % 16 == 0,
+              "stage layout");
+static_assert(offsetof(RowCoef, kl) % 16 == 0 && offsetof(RowCoef, h) % 16 == 0, "row data layout");
 
 // ---------------------------------------------------------------- PTX helpers
 
@@ -412,7 +427,7 @@ __device__ __forceinline__ float magic_out(int b)
 // Pass 1: unpack the old codes, accumulate the two column sums and leave
 // per-warp partials in red.  B = 4, 6, 8: every row has B
 // bits (GDN); B = 0: per-row widths (KDA).
-template <int B, int SB, bool ACC = true>
+template <int B, int SB, bool FIT, bool ACC = true>
 __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -425,7 +440,7 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
-        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + 16 * B * i, cg, z[ii]);
+        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
         else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
         if constexpr (ACC) {
             const float4 kl = R.kl[i];
@@ -453,13 +468,39 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
     }
 }
 
+// Per column (threads 0..127), one tile after pass 2 wrote its partial sums:
+// the refitted factor c_j <- c_j sum_i A_i z'_ij w_ij / sum_i B_i z'_ij^2
+// (= sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2 with v_ij = s'_i r_i z'_ij and
+// X_ij = c_j e~_i w_ij), stored into that tile's page; a column whose codes
+// are all zero keeps its factor.
+template <int SB>
+__device__ __forceinline__ void fit_finish(Smem &sm, int parity)
+{
+    if (!sm.fit_pending[parity]) return;
+    const int j = threadIdx.x;
+    const int at = ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3);
+    float num = 0.0f, den = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        num += sm.red2[w * 256 + at];
+        den += sm.red2[w * 256 + 128 + at];
+    }
+    const float c_old = sm.fitc[j];
+    const float c_new = den > 0.0f ? c_old * __fdiv_rn(num, den) : c_old;
+    if (!isfinite(c_new)) atomicOr(&sm.flags, kErrNonFinite);
+    reinterpret_cast<float *>(sm.fit_page[parity] + SB * kD)[j] = c_new;
+}
+
 // Per column (threads 0..127): v_old, u, y, u / c.  The write-back takes
 // u / c from the readout's buffer (prefetched into the stage's v) instead.
-template <int MODE>
+template <int MODE, int SB, bool FIT>
 __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const RowCoef &R,
                                                 const DecodeIO &io, int tile, float beta)
 {
     const int j = threadIdx.x;
+    // the column factors this tile's codes are read and taken with
+    const float cj = FIT ? reinterpret_cast<const float *>(S.page + SB * kD)[j] : S.c[j];
+    if (FIT && MODE != kReadout) sm.fitc[j] = cj;
     if (MODE == kWriteback) {
         sm.ut[j] = S.v[j];
         return;
@@ -471,7 +512,6 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
         vz += sm.red[w * 256 + at];
         yz += sm.red[w * 256 + 128 + at];
     }
-    const float cj = S.c[j];
     const float u = beta * (S.v[j] - cj * vz);
     const float kq = (R.kqp[0] + R.kqp[1]) + (R.kqp[2] + R.kqp[3]);
     const float yj = fmaf(u, kq, cj * yz);
@@ -484,7 +524,7 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
 
 // Per row (threads 128..255) of the next tile: decayed scale e_i and the
 // coefficients both passes need; warp 4 also forms k.q.
-template <int KIND, int SB, int MODE>
+template <int KIND, int SB, int MODE, bool FIT>
 __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, int s)
 {
     const int r = threadIdx.x - kD;
@@ -507,6 +547,10 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     R.kl[r] = make_float4(ka, ka, la, la);
     R.h[r] = dropped ? kr : hq;
     R.mrq[r] = (dropped ? 1.0f : e) * S.inv_rq[r];
+    if (FIT) {
+        const float wr = sm.stage_w[s][r] * rr;
+        R.fb[r] = wr * wr;
+    }
     R.off[r] = S.row_off[r];
     R.bits[r] = S.row_bits[r];
     const uint32_t bal = __ballot_sync(0xffffffffu, dropped);
@@ -521,7 +565,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
 // groups of the half-warp through shared memory), new scale, requantise,
 // store codes and scales to the page in global memory.
-template <int B, int SB>
+template <int B, int SB, bool FIT>
 __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -614,6 +658,11 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
                     atomicOr(&sm.flags, kErrNonFinite);
                 }
                 reinterpret_cast<float *>(page)[i] = snew;
+                if (FIT) {
+                    // A = w^2 r e~ s' = (w r)^2 q_b mrq s', since mrq = e~ / (r q_b)
+                    sm.rowA[i] = ((R.fb[i] * qb) * mrq) * snew;
+                    sm.rowB[i] = (R.fb[i] * snew) * snew;
+                }
             } else {
                 // binary16 scale: s16 = half(a / q_b); the codes are rounded from
                 // mu / s16 = w (e / r) / s16 = w mrq q_b / s16
@@ -626,6 +675,11 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
                 // rounds to at most q_b (q_b <= 127); only a subnormal s16 can round further down
                 clip = sf < s && sf < 6.103515625e-05f;
                 reinterpret_cast<__half *>(page)[i] = s16;
+                if (FIT) {
+                    const float sv = sf <= 65504.0f ? sf : 0.0f;
+                    sm.rowA[i] = ((R.fb[i] * qb) * mrq) * sv;
+                    sm.rowB[i] = (R.fb[i] * sv) * sv;
+                }
             }
             sm.rowinv[i] = inv;
         }
@@ -637,6 +691,13 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
     const float4 ia = *reinterpret_cast<const float4 *>(&sm.rowinv[i0]);
     const float4 ib = *reinterpret_cast<const float4 *>(&sm.rowinv[i0 + 4]);
     const float invs[8] = {ia.x, ia.y, ia.z, ia.w, ib.x, ib.y, ib.z, ib.w};
+    // column fit: per-column sums of A_i z'_ij w_ij and B_i z'_ij^2 over this thread's rows
+    float2 fnum[4], fden[4];
+    if (FIT) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) fnum[p] = fden[p] = make_float2(0.0f, 0.0f);
+    }
+    uint8_t *rows = page + SB * kD + (FIT ? kFitBytes : 0);
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
@@ -665,9 +726,30 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
             }
             bits[2 * p] = __float_as_uint(t.x);
             bits[2 * p + 1] = __float_as_uint(t.y);
+            if (FIT) {
+                // z' = t - mg exactly (the new code); A z' w and B z'^2 into the column sums
+                const float2 zq = fadd2(t, make_float2(-mg, -mg));
+                const float A = sm.rowA[i], Bc = sm.rowB[i];
+                fnum[p] = ffma2(make_float2(A, A), fmul2(zq, z[ii][p]), fnum[p]);
+                fden[p] = ffma2(make_float2(Bc, Bc), fmul2(zq, zq), fden[p]);
+            }
         }
-        if (B != 0) Codec<B == 0 ? 8 : B>::store(page + SB * kD + 16 * B * i, cg, bits);
+        if (B != 0) Codec<B == 0 ? 8 : B>::store(rows + 16 * B * i, cg, bits);
         else store_any(b, page + R.off[i], cg, bits);
+    }
+    if (FIT) {
+        // per-warp partials, laid out as pass 1's column sums (half 0 numerators, half 1 denominators)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            fnum[p] = fadd2(fnum[p], make_float2(__shfl_xor_sync(0xffffffffu, fnum[p].x, 16),
+                                                 __shfl_xor_sync(0xffffffffu, fnum[p].y, 16)));
+            fden[p] = fadd2(fden[p], make_float2(__shfl_xor_sync(0xffffffffu, fden[p].x, 16),
+                                                 __shfl_xor_sync(0xffffffffu, fden[p].y, 16)));
+        }
+        const float2 *src = rgl == 0 ? fnum : fden;
+        float *dst = &sm.red2[warp * 256 + rgl * 128 + cg * 4];
+        *reinterpret_cast<float4 *>(dst) = make_float4(src[0].x, src[0].y, src[1].x, src[1].y);
+        *reinterpret_cast<float4 *>(dst + 64) = make_float4(src[2].x, src[2].y, src[3].x, src[3].y);
     }
 }
 
@@ -713,6 +795,7 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
 {
     Stage &S = sm.st[s];
     sm.stage_page[s] = t.page;
+    sm.stage_w[s] = p.t.w + static_cast<size_t>(t.h) * kD;
     // a page larger than a stage is a GDN FP16 pivot head, advanced by its own kernel
     const bool mine = t.valid && t.bytes <= static_cast<uint32_t>(kMaxPage);
     sm.stage_valid[s] = mine;
@@ -807,7 +890,7 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
 // A stage is last read before the second barrier of its tile (pass 2 reads
 // only registers and the row data); thread 96 refills it after the first
 // barrier of the next tile.
-template <int KIND, int SB, int MODE>
+template <int KIND, int SB, int MODE, bool FIT>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
     extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -819,6 +902,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
 
     if (tid == 0) {
         sm.flags = 0;
+        sm.fit_pending[0] = sm.fit_pending[1] = 0;
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
         fence_mbar_init();
         fence_proxy_async_smem();
@@ -844,7 +928,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
     bool timed_out = false;
     if (tid >= kD) {
         // warp-uniform outcome: row_setup's shuffles need every lane
-        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB, MODE>(sm, sm.st[0], sm.rc[0], 0);
+        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB, MODE, FIT>(sm, sm.st[0], sm.rc[0], 0);
         else timed_out = true;
     }
     timed_out = __syncthreads_or(timed_out) != 0;
@@ -863,10 +947,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         float2 z[8][4];
         constexpr bool kAcc = MODE != kWriteback;
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0, SB, kAcc>(sm, S, R, z);  // per-row widths (and KDA pivot rows)
-            else if (b == 8) pass1<8, SB, kAcc>(sm, S, R, z);
-            else if (b == 6) pass1<6, SB, kAcc>(sm, S, R, z);
-            else pass1<4, SB, kAcc>(sm, S, R, z);
+            if (KIND == STQ_KDA) pass1<0, SB, FIT, kAcc>(sm, S, R, z);  // per-row widths (and KDA pivot rows)
+            else if (b == 8) pass1<8, SB, FIT, kAcc>(sm, S, R, z);
+            else if (b == 6) pass1<6, SB, FIT, kAcc>(sm, S, R, z);
+            else pass1<4, SB, FIT, kAcc>(sm, S, R, z);
         }
         cp_async_wait<1>();
         __syncthreads();
@@ -881,21 +965,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         bool tout = false;
         if (tid < kD) {
-            if (valid) column_epilogue<MODE>(sm, S, R, io, tile, sm.beta[s]);
+            constexpr bool kFits = FIT && MODE != kReadout;
+            if (kFits) fit_finish<SB>(sm, (i + 1) & 1);  // the previous tile's factors
+            if (valid) column_epilogue<MODE, SB, FIT>(sm, S, R, io, tile, sm.beta[s]);
+            if (kFits && tid == 0) {
+                sm.fit_page[i & 1] = R.page;
+                sm.fit_pending[i & 1] = valid;
+            }
         } else if (tile + G < tiles) {
             const int sn = (i + 1) % kStages;
             if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)))
-                row_setup<KIND, SB, MODE>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
+                row_setup<KIND, SB, MODE, FIT>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
             else
                 tout = true;
         }
         timed_out = __syncthreads_or(tout) != 0;
         if (valid && MODE != kReadout) {
-            if (KIND == STQ_KDA) pass2<0, SB>(sm, R, z);
-            else if (b == 8) pass2<8, SB>(sm, R, z);
-            else if (b == 6) pass2<6, SB>(sm, R, z);
-            else pass2<4, SB>(sm, R, z);
+            if (KIND == STQ_KDA) pass2<0, SB, FIT>(sm, R, z);
+            else if (b == 8) pass2<8, SB, FIT>(sm, R, z);
+            else if (b == 6) pass2<6, SB, FIT>(sm, R, z);
+            else pass2<4, SB, FIT>(sm, R, z);
         }
+    }
+    if (FIT && MODE != kReadout) {
+        __syncthreads();  // the last tile's partial sums are in
+        if (!timed_out && tid < kD) fit_finish<SB>(sm, (i + 1) & 1);
     }
     cp_async_wait<0>();  // no copy may land in this CTA's shared memory after it exits
 
@@ -916,7 +1010,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
 
 constexpr int kMaxDevices = 64;
 
-template <int KIND, int SB, int MODE>
+template <int KIND, int SB, int MODE, bool FIT>
 cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
     // per device: SM count, and the dynamic shared-memory opt-in of this kernel
@@ -930,23 +1024,31 @@ cudaError_t launch(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
         int n = 0;
         e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(decode_kernel<KIND, SB, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        e = cudaFuncSetAttribute(decode_kernel<KIND, SB, MODE, FIT>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         sms[dev] = n > 0 ? n : 148;
     }
     const int tiles = io.n * p.H;
     const int grid = tiles < 2 * sms[dev] ? tiles : 2 * sms[dev];
-    decode_kernel<KIND, SB, MODE><<<grid, kThreads, smem, stream>>>(p, io, tiles);
+    decode_kernel<KIND, SB, MODE, FIT><<<grid, kThreads, smem, stream>>>(p, io, tiles);
     count_launch();
     return cudaGetLastError();
+}
+
+template <int MODE, bool FIT>
+cudaError_t launch_fit(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
+{
+    if (p.scale_bytes == 2)
+        return p.kind == STQ_KDA ? launch<STQ_KDA, 2, MODE, FIT>(p, io, stream)
+                                 : launch<STQ_GDN, 2, MODE, FIT>(p, io, stream);
+    return p.kind == STQ_KDA ? launch<STQ_KDA, 4, MODE, FIT>(p, io, stream)
+                             : launch<STQ_GDN, 4, MODE, FIT>(p, io, stream);
 }
 
 template <int MODE>
 cudaError_t launch_mode(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
-    if (p.scale_bytes == 2)
-        return p.kind == STQ_KDA ? launch<STQ_KDA, 2, MODE>(p, io, stream) : launch<STQ_GDN, 2, MODE>(p, io, stream);
-    return p.kind == STQ_KDA ? launch<STQ_KDA, 4, MODE>(p, io, stream) : launch<STQ_GDN, 4, MODE>(p, io, stream);
+    return p.fit ? launch_fit<MODE, true>(p, io, stream) : launch_fit<MODE, false>(p, io, stream);
 }
 
 }  // namespace

@@ -13,7 +13,8 @@ namespace stq {
 constexpr int kD = 128;            // d_k = d_v
 constexpr int kScaleBytes = 4 * kD; // fp32 scales at the start of a page
 constexpr int kPageAlign = 128;    // pages are padded to this many bytes
-constexpr int kMaxStagedPage = kScaleBytes + 16 * 8 * kD;  // largest page the fused kernel stages (8 bits per row)
+constexpr int kMaxStagedPage = kScaleBytes + 4 * kD + 16 * 8 * kD;  // largest page the fused kernel stages
+                                                                    // (8 bits per row, fitted column factors)
 constexpr size_t kStaticScratchFloats = size_t(1) << 20;  // built-in u~ buffer: 4 MiB, 8192 tiles
 
 // device error word bits
@@ -27,9 +28,11 @@ constexpr uint32_t kErrTimeout = 4u;
 //   row_off[H][128] byte offset of row i inside the page (scales come first)
 //   row_bits[H][128]
 //   r[H][128], c[H][128]
+//   w[H][128]       row weights of the column fit
 //   block[H][kHeadBlock]: r, c, 1 / (r q_b), row_off, row_bits of one head
 //                  side by side, so that the decode kernel fetches them with one copy
 constexpr int kHeadBlock = 2048;  // 512 (r) + 512 (c) + 512 (1 / (r q_b)) + 256 (row_off) + 128 (row_bits), padded
+constexpr int kFitBytes = 4 * kD;  // a fitted page's own column factors (fp32), after the scales
 struct Tables {
     const uint32_t *head_off;
     const uint32_t *page_bytes;
@@ -37,6 +40,7 @@ struct Tables {
     const uint8_t *row_bits;
     const float *r;
     const float *c;
+    const float *w;
     const uint8_t *block;
 };
 
@@ -48,6 +52,7 @@ struct PoolView {
     int scale_bytes;     // bytes per row scale: 4 (fp32) or 2 (binary16); 0 in a raw pool
     int raw_bits;        // 16 or 32 in a raw pool (every unit), else 0
     int pivots;          // nonzero if 16-bit (FP16 pivot) units sit among quantized ones
+    int fit;             // nonzero: pages carry column factors refitted at every quantisation
     Tables t;
     uint32_t *err;
 };

@@ -32,10 +32,15 @@ __device__ __forceinline__ uint8_t *tile_page(const PoolView &p, int req, int sl
 
 // fp32 state -> packed page: mu = fl32(S / (r c)) (fp64 quotient), s = fl32(max|mu| / q_b),
 // z = clip(rint(fl32(mu / s)), -q_b, q_b).  A 16-bit row is an FP16 pivot: its scale
-// slot holds 1 and it stores mu rounded once to binary16.  One warp per row.
+// slot holds 1 and it stores mu rounded once to binary16.  With fitted column
+// factors the codes are taken with the table's c, then every column is refitted
+// in fp64, c_j = sum_i w_i^2 v_ij S_ij / sum_i w_i^2 v_ij^2 with v_ij = s_i r_i z_ij
+// (each term formed in the oracle's operation order), and stored in the page.
+// One warp per row.
 __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t *req_idx,
                                                        const int32_t *slot_idx, const float *state)
 {
+    __shared__ double fit_sum[8][2][kD];  // per-warp column sums of the fit (num, den)
     const int tile = blockIdx.x;
     const int ni = tile / p.H, h = tile - ni * p.H;
     const int req = req_idx[ni], slot = slot_idx[ni];
@@ -48,6 +53,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float4 c4 = *reinterpret_cast<const float4 *>(p.t.c + h * kD + lane * 4);
     const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
+    const float *wrow = p.t.w + static_cast<size_t>(h) * kD;
+    double fnum[4] = {0.0, 0.0, 0.0, 0.0}, fden[4] = {0.0, 0.0, 0.0, 0.0};
     bool bad = false;
     for (int i = warp; i < kD; i += 8) {
         const int b = p.t.row_bits[h * kD + i];
@@ -111,8 +118,36 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
             if (p.scale_bytes == 2) reinterpret_cast<__half *>(page)[i] = s16;
             else reinterpret_cast<float *>(page)[i] = s;
         }
+        if (p.fit) {
+            const double wi = static_cast<double>(wrow[i]);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const double v = static_cast<double>(s) * r * static_cast<double>(static_cast<int>(code[t]));
+                fnum[t] += wi * wi * v * static_cast<double>(x[t]);
+                fden[t] += wi * wi * v * v;
+            }
+        }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kErrNonFinite);
+    if (p.fit) {  // uniform over the CTA
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            fit_sum[warp][0][lane * 4 + t] = fnum[t];
+            fit_sum[warp][1][lane * 4 + t] = fden[t];
+        }
+        __syncthreads();
+        if (threadIdx.x < kD) {
+            const int j = threadIdx.x;
+            double num = 0.0, den = 0.0;
+            for (int w = 0; w < 8; ++w) {
+                num += fit_sum[w][0][j];
+                den += fit_sum[w][1][j];
+            }
+            const float cn = den > 0.0 ? static_cast<float>(num / den) : p.t.c[h * kD + j];
+            if (!isfinite(cn)) atomicOr(p.err, kErrNonFinite);
+            reinterpret_cast<float *>(page + p.scale_bytes * kD)[j] = cn;
+        }
+    }
 }
 
 // packed page -> fp32 reconstruction fl32(((s r) c) z) computed in fp64 (z: the binary16
@@ -130,7 +165,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
     const uint8_t *page = tile_page(p, req, slot, h);
     float *S = state + static_cast<size_t>(tile) * kD * kD;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float4 c4 = *reinterpret_cast<const float4 *>(p.t.c + h * kD + lane * 4);
+    // the column factors: the page's own when they are fitted, else the table's
+    const float4 c4 = *reinterpret_cast<const float4 *>((p.fit ? reinterpret_cast<const float *>(page + p.scale_bytes * kD)
+                                                                : p.t.c + h * kD) + lane * 4);
     const float cj[4] = {c4.x, c4.y, c4.z, c4.w};
     for (int i = warp; i < kD; i += 8) {
         const int b = p.t.row_bits[h * kD + i];

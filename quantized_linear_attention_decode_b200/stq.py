@@ -16,6 +16,7 @@ LIB_PATH = os.path.join(_PKG, "libstq.so")
 
 STQ_GDN, STQ_KDA = 0, 1
 STQ_SCALE_F16 = 1  # desc flag: per-row scales stored as IEEE binary16
+STQ_FIT_COLUMNS = 2  # desc flag: per-page column factors refitted at every quantisation
 STQ_ALLOC_DP, STQ_ALLOC_LAGRANGE = 0, 1  # bit allocation methods
 STATUS = {0: "STQ_OK", 1: "STQ_ERR_ARG", 2: "STQ_ERR_OOM", 3: "STQ_ERR_CUDA", 4: "STQ_ERR_INDEX",
           5: "STQ_ERR_NONFINITE", 6: "STQ_ERR_UNSUPPORTED", 7: "STQ_ERR_TIMEOUT"}
@@ -41,7 +42,7 @@ class _Desc(C.Structure):
     _fields_ = [("kind", C.c_int32), ("num_requests", C.c_int32), ("num_slots", C.c_int32),
                 ("num_heads", C.c_int32), ("d_k", C.c_int32), ("d_v", C.c_int32),
                 ("unit_bits", C.c_void_p), ("row_factor", C.c_void_p), ("col_factor", C.c_void_p),
-                ("flags", C.c_uint32)]
+                ("flags", C.c_uint32), ("row_weight", C.c_void_p)]
 
 
 _lib = None
@@ -120,13 +121,14 @@ def _dev(t, dtype, shape=None, name="tensor"):
     return C.c_void_p(t.data_ptr())
 
 
-def _desc(kind, R, S, H, unit_bits, row_factor, col_factor, keep, flags=0):
+def _desc(kind, R, S, H, unit_bits, row_factor, col_factor, keep, flags=0, row_weight=None):
     ub = np.ascontiguousarray(unit_bits, np.uint8)
     rf = None if row_factor is None else np.ascontiguousarray(row_factor, np.float32)
     cf = None if col_factor is None else np.ascontiguousarray(col_factor, np.float32)
-    keep.extend([ub, rf, cf])
+    rw = None if row_weight is None else np.ascontiguousarray(row_weight, np.float32)
+    keep.extend([ub, rf, cf, rw])
     ptr = lambda a: None if a is None else a.ctypes.data  # noqa: E731
-    return _Desc(int(kind), int(R), int(S), int(H), 128, 128, ptr(ub), ptr(rf), ptr(cf), int(flags))
+    return _Desc(int(kind), int(R), int(S), int(H), 128, 128, ptr(ub), ptr(rf), ptr(cf), int(flags), ptr(rw))
 
 
 class Pool:
@@ -162,9 +164,10 @@ class Pool:
 
 
 def stq_pool_create(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
-                    col_factor=None, flags=0) -> Pool:
+                    col_factor=None, flags=0, row_weight=None) -> Pool:
     keep = []
-    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags)
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags,
+              row_weight)
     h = C.c_void_p()
     _check(load().stq_pool_create(C.byref(d), C.byref(h)))
     return Pool(h, kind, num_requests, num_slots, num_heads, unit_bits, flags)
@@ -181,9 +184,10 @@ def stq_pool_bytes(pool: Pool):
 
 
 def stq_desc_bytes(kind, num_requests, num_slots, num_heads, unit_bits, row_factor=None,
-                   col_factor=None, flags=0):
+                   col_factor=None, flags=0, row_weight=None):
     keep = []
-    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags)
+    d = _desc(kind, num_requests, num_slots, num_heads, unit_bits, row_factor, col_factor, keep, flags,
+              row_weight)
     a, b = C.c_size_t(), C.c_size_t()
     _check(load().stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)))
     return a.value, b.value

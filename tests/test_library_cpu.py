@@ -91,6 +91,19 @@ def test_desc_bytes_formats():
     assert s32 == 2 * s16
 
 
+def test_desc_bytes_fitted_columns():
+    """Fitted column factors add 128 fp32 values to every page; row weights must be > 0."""
+    bits = np.array([4, 6, 8, 6], np.uint8)
+    _, plain = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits)
+    _, fit = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits, flags=stq.STQ_FIT_COLUMNS)
+    assert fit - plain == 4 * 512
+    w = np.ones(4 * 128, np.float32)
+    w[7] = 0.0
+    with pytest.raises(stq.StqError) as e:
+        stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits, flags=stq.STQ_FIT_COLUMNS, row_weight=w)
+    assert e.value.status == stq.STQ_ERR_ARG
+
+
 def test_desc_bytes_pivot_pool():
     """16-bit units among quantized ones are FP16 pivots: every page keeps its scale
     section, a pivot head holds 128 rows of 256 B."""
@@ -107,7 +120,9 @@ def test_desc_bytes_pivot_pool():
     ([32, 16, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),  # two raw widths
     ([32, 8, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),   # fp32 units among quantized ones
     ([16, 16, 16, 16], 1, "STQ_ERR_ARG"),          # a raw pool has no scales
-    ([6, 6, 6, 6], 2, "STQ_ERR_ARG"),              # unknown flag
+    ([6, 6, 6, 6], 4, "STQ_ERR_ARG"),              # unknown flag
+    ([16, 6, 8, 6], 2, "STQ_ERR_UNSUPPORTED"),     # fitted column factors with FP16 pivots
+    ([16, 16, 16, 16], 2, "STQ_ERR_ARG"),          # a raw pool has no scales or factors
     ([6, 12, 6, 6], 0, "STQ_ERR_ARG"),
 ])
 def test_desc_format_validation(ub, flags, status):
@@ -119,7 +134,7 @@ def test_desc_format_validation(ub, flags, status):
 def test_unsupported_head_dim():
     L = stq.load()
     ub = np.array([6], np.uint8)
-    d = stq._Desc(0, 1, 1, 1, 64, 64, ub.ctypes.data, None, None, 0)
+    d = stq._Desc(0, 1, 1, 1, 64, 64, ub.ctypes.data, None, None, 0, None)
     a, b = C.c_size_t(), C.c_size_t()
     assert L.stq_desc_bytes(C.byref(d), C.byref(a), C.byref(b)) == stq.STQ_ERR_UNSUPPORTED
 
