@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--no-sweep", action="store_true", help="skip the serving-pool sweep")
     ap.add_argument("--no-layer-loop", action="store_true", help="skip the 48-layer graph comparison")
+    ap.add_argument("--no-drift", action="store_true", help="skip the long-generation drift record")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     return ap.parse_args()
@@ -394,6 +395,9 @@ def run_ours(args, rank: int, world: int):
     loop = None
     if rank == 0 and world == 1 and not args.no_layer_loop:
         loop = layer_loop(stq, flush)
+    drift_log = None
+    if rank == 0 and world == 1 and not args.no_drift:
+        drift_log = drift(stq)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -425,6 +429,7 @@ def run_ours(args, rank: int, world: int):
         "clocks": sampler.summary(),
         "pool_sweep": sweep,
         "layer_loop": loop,
+        "drift": drift_log,
     }
     print(json.dumps(line), flush=True)
 
@@ -530,6 +535,60 @@ def layer_loop(stq, flush, layers: int = 48, R: int = 64, reps: int = 20):
         stq.stq_pool_check(p)
         p.close()
     torch.cuda.empty_cache()
+    return out
+
+
+def drift(stq, steps: int = 8192, every: int = 512, tokens: int = 256):
+    """Long-generation drift: 32 requests x 32 heads, alpha ~ U(0.95, 0.9999),
+    GDN at INT4 / INT6 / INT8 and KDA at 6-bit mixed widths (decay per row in
+    the same range), each advanced `steps` tokens next to the unquantized fp32
+    recurrence (a raw fp32 pool) on the same inputs; every `every` steps the
+    relative state error ||S^ - S||_F / ||S||_F and readout error
+    ||y^ - y|| / ||y|| per (request, head) are recorded (mean and max).  The
+    inputs of `tokens` distinct steps are cycled."""
+    import dataclasses
+    import torch
+    cases = [(f"gdn_int{b}", synth.make_workload(5, bits=b)) for b in (4, 6, 8)]
+    kda = synth.make_workload(3, R=32, H=32)
+    cases.append(("kda_mixed6", dataclasses.replace(kda, decay_range=(0.95, 0.9999), name="drift_kda_mixed6")))
+    out = {"steps": steps, "every": every, "tokens_cycled": tokens, "requests": 32, "heads": 32, "cases": {}}
+    for name, wl in cases:
+        n_units = wl.H if wl.kind == synth.GDN else wl.H * 128
+        ctl = dataclasses.replace(wl, unit_bits=np.full(n_units, 32, np.uint8))
+        pq = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
+        pf = stq.stq_pool_create(ctl.kind, ctl.R, ctl.S, ctl.H, ctl.unit_bits)
+        req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
+        slot = torch.zeros(wl.R, dtype=torch.int32, device="cuda")
+        xs = []
+        for t in range(tokens):
+            inp = wl.step_inputs(t)
+            xs.append([torch.from_numpy(inp[k]).cuda() for k in ("q", "k", "v", "beta", "gate")])
+        yq = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
+        yf = torch.empty_like(yq)
+        Sq = torch.empty((wl.R, wl.H, 128, 128), dtype=torch.float32, device="cuda")
+        Sf = torch.empty_like(Sq)
+        rec = {"state_rel_err_mean": [], "state_rel_err_max": [], "y_rel_err_mean": [], "y_rel_err_max": []}
+        for t in range(steps):
+            x = xs[t % tokens]
+            stq.stq_decode_step(pq, req, slot, *x, yq)
+            stq.stq_decode_step(pf, req, slot, *x, yf)
+            if (t + 1) % every == 0:
+                stq.stq_dequantize_state(pq, req, slot, Sq)
+                stq.stq_dequantize_state(pf, req, slot, Sf)
+                es = (torch.linalg.vector_norm(Sq - Sf, dim=(2, 3)) /
+                      torch.linalg.vector_norm(Sf, dim=(2, 3)).clamp_min(1e-30))
+                ey = torch.linalg.vector_norm(yq - yf, dim=2) / torch.linalg.vector_norm(yf, dim=2).clamp_min(1e-30)
+                rec["state_rel_err_mean"].append(float(es.mean()))
+                rec["state_rel_err_max"].append(float(es.max()))
+                rec["y_rel_err_mean"].append(float(ey.mean()))
+                rec["y_rel_err_max"].append(float(ey.max()))
+        stq.stq_pool_check(pq)
+        stq.stq_pool_check(pf)
+        out["cases"][name] = rec
+        pq.close()
+        pf.close()
+        del xs, Sq, Sf
+        torch.cuda.empty_cache()
     return out
 
 
