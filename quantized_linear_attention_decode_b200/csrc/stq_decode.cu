@@ -48,6 +48,7 @@ constexpr int kFused = 0;      // the whole step (one state traversal)
 constexpr int kReadout = 1;    // steps 1-3: y and u~; the page is only read
 constexpr int kWriteback = 2;  // steps 4-7 given u~: requantise and pack in place
 constexpr int kStages = 4;
+constexpr int kRedStride = 288;  // floats per warp in red: 256 column partials, or the padded row-max exchange
 constexpr int kMaxPage = kMaxStagedPage;               // 16896: every row at 8 bits
 constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
 
@@ -83,7 +84,7 @@ struct __align__(16) RowCoef {
 struct __align__(128) Smem {
     Stage st[kStages];
     RowCoef rc[2];
-    float red[2048];   // column partial sums [8 warps][v, y][128]; then row-max partials
+    float red[8 * kRedStride];  // per warp: column partial sums [v, y][128]; then row-max partials
     float rowinv[kD];  // per-row quantisation multiplier (pass 2)
     float red2[2048];  // column fit partial sums [8 warps][num, den][128], finished in the next tile
     float rowA[kD], rowB[kD];  // column fit row coefficients of pass 2: A = fa s', B = fb s'^2
@@ -462,10 +463,19 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
         // half 0 keeps the v-sums, half 1 the y-sums; column j of a sum sits at
         // ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3) (conflict-free 16-byte stores)
         const float2 *src = rgl == 0 ? av : ay;
-        float *dst = &sm.red[warp * 256 + rgl * 128 + cg * 4];
+        float *dst = &sm.red[warp * kRedStride + rgl * 128 + cg * 4];
         *reinterpret_cast<float4 *>(dst) = make_float4(src[0].x, src[0].y, src[1].x, src[1].y);
         *reinterpret_cast<float4 *>(dst + 64) = make_float4(src[2].x, src[2].y, src[3].x, src[3].y);
     }
+}
+
+// Column handled by epilogue thread t (0..127): a permutation under which the
+// 32 lanes of a warp read 32 distinct banks of the column partial sums (whose
+// column j sits at ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3)).
+__device__ __forceinline__ int epilogue_column(int t)
+{
+    const int w = t >> 5, lane = t & 31;
+    return ((((w >> 1) << 3) + (lane >> 2)) << 3) | ((w & 1) << 2) | (lane & 3);
 }
 
 // Per column (threads 0..127), one tile after pass 2 wrote its partial sums:
@@ -477,7 +487,7 @@ template <int SB>
 __device__ __forceinline__ void fit_finish(Smem &sm, int parity)
 {
     if (!sm.fit_pending[parity]) return;
-    const int j = threadIdx.x;
+    const int j = epilogue_column(threadIdx.x);
     const int at = ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3);
     float num = 0.0f, den = 0.0f;
 #pragma unroll
@@ -497,7 +507,7 @@ template <int MODE, int SB, bool FIT>
 __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const RowCoef &R,
                                                 const DecodeIO &io, int tile, float beta)
 {
-    const int j = threadIdx.x;
+    const int j = epilogue_column(threadIdx.x);
     // the column factors this tile's codes are read and taken with
     const float cj = FIT ? reinterpret_cast<const float *>(S.page + SB * kD)[j] : S.c[j];
     if (FIT && MODE != kReadout) sm.fitc[j] = cj;
@@ -509,8 +519,8 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     float vz = 0.0f, yz = 0.0f;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) {
-        vz += sm.red[w * 256 + at];
-        yz += sm.red[w * 256 + 128 + at];
+        vz += sm.red[w * kRedStride + at];
+        yz += sm.red[w * kRedStride + 128 + at];
     }
     const float u = beta * (S.v[j] - cj * vz);
     const float kq = (R.kqp[0] + R.kqp[1]) + (R.kqp[2] + R.kqp[3]);
@@ -618,10 +628,12 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
         mx[ii] = fmaxf(m, fabsf(z[ii][3].y));
     }
     // row maxima: this thread's 8 partials -> shared; lane (rgl, cg) then reduces row
-    // 8 rg + (cg & 7) over the 8 column groups of half cg >> 3 (conflict-free layout)
-    float *rm = &sm.red[warp * 256];
+    // 8 rg + (cg & 7) over the 8 column groups of half cg >> 3.  Column group m of a half
+    // sits 36 floats from group m - 1, so that both the 16-byte stores (each quarter
+    // warp on distinct banks) and the scalar loads are free of bank conflicts.
+    float *rm = &sm.red[warp * kRedStride];
     {
-        float4 *dst = reinterpret_cast<float4 *>(&rm[(cg & 7) * 32 + rgl * 16 + (cg >> 3) * 8]);
+        float4 *dst = reinterpret_cast<float4 *>(&rm[(cg & 7) * 36 + rgl * 16 + (cg >> 3) * 8]);
         dst[0] = make_float4(mx[0], mx[1], mx[2], mx[3]);
         dst[1] = make_float4(mx[4], mx[5], mx[6], mx[7]);
     }
@@ -631,10 +643,10 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
     {
         const int ii = cg & 7, half = cg >> 3;
         const float *src = &rm[rgl * 16 + half * 8 + ii];
-        float m = max3(src[0], src[32], src[64]);
-        m = max3(m, src[96], src[128]);
-        m = max3(m, src[160], src[192]);
-        m = fmaxf(m, src[224]);
+        float m = max3(src[0], src[36], src[72]);
+        m = max3(m, src[108], src[144]);
+        m = max3(m, src[180], src[216]);
+        m = fmaxf(m, src[252]);
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
         if (half == 0) {
             const int i = i0 + ii;
