@@ -89,7 +89,7 @@ struct __align__(128) Smem {
     float red2[2048];  // column fit partial sums [8 warps][num, den][128], finished in the next tile
     float rowA[kD], rowB[kD];  // column fit row coefficients of pass 2: A = fa s', B = fb s'^2
     float fitc[kD];    // the column factors the tile's codes were taken with
-    float ut[kD];      // u_j / c_j
+    float ut[kD];      // u_j / c_j, column j at ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3)
     uint8_t *stage_page[kStages];
     const float *stage_w[kStages];  // the tile's head row weights (column fit)
     uint32_t stage_valid[kStages];
@@ -511,11 +511,13 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     // the column factors this tile's codes are read and taken with
     const float cj = FIT ? reinterpret_cast<const float *>(S.page + SB * kD)[j] : S.c[j];
     if (FIT && MODE != kReadout) sm.fitc[j] = cj;
+    // column j's slot in the partial sums, and in ut (columns 8 g .. 8 g + 3 of a column group
+    // g at 4 g, columns 8 g + 4 .. 8 g + 7 at 64 + 4 g: pass 2 reads them as 16-byte vectors)
+    const int at = ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3);
     if (MODE == kWriteback) {
-        sm.ut[j] = S.v[j];
+        sm.ut[at] = S.v[j];
         return;
     }
-    const int at = ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3);
     float vz = 0.0f, yz = 0.0f;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) {
@@ -528,7 +530,7 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     io.y[static_cast<size_t>(tile) * kD + j] = yj;
     const float ut = u * rcp_approx(cj);
     if (MODE == kReadout) io.u_out[static_cast<size_t>(tile) * kD + j] = ut;
-    else sm.ut[j] = ut;
+    else sm.ut[at] = ut;
     if (!isfinite(u) || !isfinite(yj)) atomicOr(&sm.flags, kErrNonFinite);
 }
 
@@ -584,8 +586,8 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
     const int i0 = (warp * 2 + rgl) * 8;
     float2 ut2[4];
     {
-        const float4 a = *reinterpret_cast<const float4 *>(&sm.ut[cg * 8]);
-        const float4 b = *reinterpret_cast<const float4 *>(&sm.ut[cg * 8 + 4]);
+        const float4 a = *reinterpret_cast<const float4 *>(&sm.ut[cg * 4]);
+        const float4 b = *reinterpret_cast<const float4 *>(&sm.ut[64 + cg * 4]);
         ut2[0] = make_float2(a.x, a.y);
         ut2[1] = make_float2(a.z, a.w);
         ut2[2] = make_float2(b.x, b.y);
@@ -827,27 +829,34 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
 // i + 3 into its stage, and the raw location {req, slot, head offset, page
 // bytes} of tile i + 5 = (request entry n5, head h5).  The small copies are
 // spread over warps 5-7, which have the least other work at this point.
+// cp.async of tile `tile`'s q, k, v (and the KDA decay), beta and alpha into stage s
+// (warps 0-3 the vectors, threads 160 and 192 the scalars); the caller commits.
+template <int KIND, int MODE>
+__device__ __forceinline__ void prefetch_vectors(Smem &sm, const DecodeIO &io, int s, int tile)
+{
+    const int t = threadIdx.x;
+    Stage &S = sm.st[s];
+    const size_t base = static_cast<size_t>(tile) * kD + 4 * (t & 31);
+    if (t < 32) {
+        if (MODE != kWriteback) cp_async16(&S.q[4 * t], io.q + base);
+    }
+    else if (t < 64) cp_async16(&S.k[4 * (t - 32)], io.k + base);
+    else if (t < 96) cp_async16(&S.v[4 * (t - 64)], io.v + base);
+    else if (t < 128) {
+        if (KIND == STQ_KDA) cp_async16(&S.g[4 * (t - 96)], io.gate + base);
+    } else if (t == 160) {
+        if (MODE != kWriteback) cp_async4(&sm.beta[s], io.beta + tile);
+    } else if (t == 192) {
+        if (KIND == STQ_GDN) cp_async4(&sm.alpha[s], io.gate + tile);
+    }
+}
+
 template <int KIND, int MODE>
 __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const DecodeIO &io, int i, int t3, int t5,
                                          int n5, int h5, int tiles)
 {
     const int t = threadIdx.x;
-    if (t3 < tiles) {
-        Stage &S = sm.st[(i + 3) % kStages];
-        const size_t base = static_cast<size_t>(t3) * kD + 4 * (t & 31);
-        if (t < 32) {
-            if (MODE != kWriteback) cp_async16(&S.q[4 * t], io.q + base);
-        }
-        else if (t < 64) cp_async16(&S.k[4 * (t - 32)], io.k + base);
-        else if (t < 96) cp_async16(&S.v[4 * (t - 64)], io.v + base);
-        else if (t < 128) {
-            if (KIND == STQ_KDA) cp_async16(&S.g[4 * (t - 96)], io.gate + base);
-        } else if (t == 160) {
-            if (MODE != kWriteback) cp_async4(&sm.beta[(i + 3) % kStages], io.beta + t3);
-        } else if (t == 192) {
-            if (KIND == STQ_GDN) cp_async4(&sm.alpha[(i + 3) % kStages], io.gate + t3);
-        }
-    }
+    if (t3 < tiles) prefetch_vectors<KIND, MODE>(sm, io, (i + 3) % kStages, t3);
     if (t5 < tiles && t >= 224 && t < 228) {
         uint32_t *dst = &sm.raw[(i + 5) & 7][t - 224];
         const void *src = t == 224 ? static_cast<const void *>(io.req_idx + n5)
@@ -858,26 +867,6 @@ __device__ __forceinline__ void prefetch(Smem &sm, const PoolView &p, const Deco
         if (t == 224) dst[4] = static_cast<uint32_t>(h5);
     }
     cp_async_commit();
-}
-
-// Synchronous fill of a stage's vectors and beta/alpha (first tiles only).
-template <int KIND, int MODE>
-__device__ __forceinline__ void fill_sync(Smem &sm, const DecodeIO &io, int s, int tile)
-{
-    const int t = threadIdx.x;
-    Stage &S = sm.st[s];
-    const size_t base = static_cast<size_t>(tile) * kD;
-    if (t < kD) {
-        if (MODE != kWriteback) S.q[t] = io.q[base + t];
-        S.k[t] = io.k[base + t];
-    } else {
-        S.v[t - kD] = io.v[base + t - kD];
-        if (KIND == STQ_KDA) S.g[t - kD] = io.gate[base + t - kD];
-    }
-    if (t == 0) {
-        sm.beta[s] = MODE != kWriteback ? io.beta[tile] : 0.0f;
-        sm.alpha[s] = KIND == STQ_GDN ? io.gate[tile] : 0.0f;
-    }
 }
 
 __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
@@ -918,25 +907,26 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
         fence_mbar_init();
         fence_proxy_async_smem();
-        for (int a = 0; a < 3; ++a) {
-            const int t = first + a * G;
-            if (t < tiles) issue<KIND>(sm, a, p, resolve(p, load_raw(p, io, t)));
-        }
-        for (int a = 3; a < 5; ++a) {
-            const int t = first + a * G;
-            if (t < tiles) {
-                const TileRaw r = load_raw(p, io, t);
-                sm.raw[a][0] = static_cast<uint32_t>(r.req);
-                sm.raw[a][1] = static_cast<uint32_t>(r.slot);
-                sm.raw[a][2] = r.hoff;
-                sm.raw[a][3] = r.bytes;
-                sm.raw[a][4] = static_cast<uint32_t>(r.h);
-            }
-        }
+    }
+    // prologue: the locations of the first five tiles (thread a loads tile a's) and,
+    // asynchronously, the vectors of the first three, all in flight together
+    if (tid < 5 && first + tid * G < tiles) {
+        const TileRaw r = load_raw(p, io, first + tid * G);
+        sm.raw[tid][0] = static_cast<uint32_t>(r.req);
+        sm.raw[tid][1] = static_cast<uint32_t>(r.slot);
+        sm.raw[tid][2] = r.hoff;
+        sm.raw[tid][3] = r.bytes;
+        sm.raw[tid][4] = static_cast<uint32_t>(r.h);
     }
     for (int a = 0; a < 3; ++a)
-        if (first + a * G < tiles) fill_sync<KIND, MODE>(sm, io, a, first + a * G);
-    __syncthreads();
+        if (first + a * G < tiles) prefetch_vectors<KIND, MODE>(sm, io, a, first + a * G);
+    cp_async_commit();
+    __syncthreads();  // barriers initialised, locations in
+    if (tid == 0)
+        for (int a = 0; a < 3; ++a)
+            if (first + a * G < tiles) issue<KIND>(sm, a, p, resolve(p, raw_from_smem(sm, a)));
+    cp_async_wait<0>();
+    __syncthreads();  // the first vectors and the stages' validity are visible
     bool timed_out = false;
     if (tid >= kD) {
         // warp-uniform outcome: row_setup's shuffles need every lane
