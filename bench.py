@@ -50,7 +50,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=2, choices=[2, 3])
+    ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4],
+                    help="2: GDN mixed 64 x 32 (default); 3: KDA 128 x 32; 4: serving pool (see --requests)")
+    ap.add_argument("--requests", type=int, default=None, help="requests of the workload (default: its own)")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--tokens", type=int, default=256, help="distinct input tokens (cycled)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
@@ -301,7 +303,7 @@ def run_ours(args, rank: int, world: int):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", dev))
-    wl = synth.make_workload(args.config, seed=shard_seed(args.seed, rank))
+    wl = synth.make_workload(args.config, seed=shard_seed(args.seed, rank), R=args.requests)
     pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
     req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
     slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
