@@ -111,9 +111,13 @@ typedef struct {
  *                    STQ_ERR_NONFINITE)
  *   with STQ_FIT_COLUMNS: then 128 fp32 column factors c_j of this page
  *   then rows i = 0..127 in order, row i holding 128 codes of b_i bits
- *   (16 * b_i bytes); code j occupies bits [j b_i, (j+1) b_i) of the row's
- *   little-endian bit string, as a b_i-bit two's complement integer in
- *   [-q_b, q_b], q_b = 2^(b_i - 1) - 1
+ *   (16 * b_i bytes), each a b_i-bit two's complement integer in
+ *   [-q_b, q_b], q_b = 2^(b_i - 1) - 1, placed in the row's little-endian
+ *   bit string (bit p is bit p % 8 of byte p / 8):
+ *     4 and 8 bits: code j at bits [j b_i, (j+1) b_i);
+ *     6 bits: codes in 16 groups of eight; group g's 48-bit string (code
+ *     8g + p at its bits [6p, 6p + 6)) is split into a 32-bit word at
+ *     bytes [4g, 4g + 4) and a 16-bit half at bytes [64 + 2g, 66 + 2g)
  *   zero padding up to a multiple of 128 bytes.
  * The pages of heads 0..H-1 follow each other inside a slot; slots are
  * ordered [request][slot].  The state the page stands for is

@@ -58,9 +58,9 @@ def lib():
         L.orc_step_unit_w.argtypes = [C.c_int, C.c_int, P, P, P, P, C.c_int, P, P, P, P, P,
                                       C.c_float, P, P, P]
         L.orc_get_code.restype = C.c_int32
-        L.orc_get_code.argtypes = [P, C.c_int, C.c_int]
+        L.orc_get_code.argtypes = [P, C.c_int, C.c_int, C.c_int]
         L.orc_put_code.restype = None
-        L.orc_put_code.argtypes = [P, C.c_int, C.c_int, C.c_int32]
+        L.orc_put_code.argtypes = [P, C.c_int, C.c_int, C.c_int, C.c_int32]
         L.orc_quantize_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P, P]
         L.orc_dequantize_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P]
         L.orc_step_unit.argtypes = [C.c_int, C.c_int, P, P, P, P, P, P, P, P, C.c_float, P, P, P]
@@ -125,14 +125,15 @@ def double_to_half(x: float) -> int:
     return int(lib().orc_double_to_half(float(x)))
 
 
-def get_code(row: np.ndarray, b: int, j: int) -> int:
+def get_code(row: np.ndarray, b: int, j: int, dv: int = 128) -> int:
+    """Code j of a packed row of dv codes of b bits."""
     row = _u8(row)
-    return int(lib().orc_get_code(_p(row), b, j))
+    return int(lib().orc_get_code(_p(row), b, dv, j))
 
 
-def put_code(row: np.ndarray, b: int, j: int, z: int) -> None:
+def put_code(row: np.ndarray, b: int, j: int, z: int, dv: int = 128) -> None:
     assert row.dtype == np.uint8 and row.flags.c_contiguous
-    lib().orc_put_code(_p(row), b, j, int(z))
+    lib().orc_put_code(_p(row), b, dv, j, int(z))
 
 
 def quantize_unit(bits, r, c, S, *, with_quot: bool = False, fmt: int = FMT_F32, w=None):

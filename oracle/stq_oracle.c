@@ -70,10 +70,16 @@
  *   bytes [0, 4 dk)        fp32 scales s_0 .. s_{dk-1} (little-endian);
  *                          [0, 2 dk) binary16 scales in format 1; no scale
  *                          section in a raw unit
- *   then row i = 0..dk-1   dv codes of b_i bits each, dv * b_i / 8 bytes;
- *                          code j occupies bits [j b_i, (j + 1) b_i) of the
- *                          row's little-endian bit string (bit p is bit p%8
- *                          of byte p/8), as a b_i-bit two's complement value
+ *   then row i = 0..dk-1   dv codes of b_i bits each, dv * b_i / 8 bytes, as
+ *                          b_i-bit two's complement values in the row's
+ *                          little-endian bit string (bit p is bit p%8 of byte
+ *                          p/8): 4- and 8-bit code j at bits [j b, (j + 1) b);
+ *                          6-bit codes in groups of eight, group g (codes
+ *                          8g .. 8g+7) a 48-bit string whose bits [0, 32) are
+ *                          the 32-bit word at bits [32 g, 32 g + 32) and whose
+ *                          bits [32, 48) are the 16-bit half at bits
+ *                          [32 G + 16 g, 32 G + 16 g + 16), G = dv / 8; code
+ *                          8g + p at bits [6p, 6p + 6) of its group
  *   padding up to a multiple of 128 bytes.
  */
 #include <math.h>
@@ -124,7 +130,7 @@ static int bits_ok(int dk, int dv, const uint8_t *bits, int fmt)
         } else if (b != 4 && b != 6 && b != 8 && !(b == 16 && (fmt & ORC_FMT_PIVOT))) {
             return 0;
         }
-        if ((dv * b) % 8 != 0) return 0;
+        if ((dv * b) % 8 != 0 || (b == 6 && dv % 8 != 0)) return 0;
     }
     return 1;
 }
@@ -193,23 +199,31 @@ uint16_t orc_double_to_half(double x)
     return (uint16_t)(sign | (uint16_t)(be << 10) | (uint16_t)((int)t - 1024));
 }
 
-/* code j of a packed row, read one bit at a time, then sign-extended */
-static int32_t get_code(const uint8_t *row, int b, int j)
+/* bit index in a row of dv codes of bit t of code j (see the page format above) */
+static int code_bit(int b, int dv, int j, int t)
+{
+    if (b != 6) return j * b + t;
+    int g = j / 8, q = 6 * (j % 8) + t; /* bit q of group g's 48-bit string */
+    return q < 32 ? 32 * g + q : 32 * (dv / 8) + 16 * g + (q - 32);
+}
+
+/* code j of a packed row of dv codes, read one bit at a time, then sign-extended */
+static int32_t get_code(const uint8_t *row, int b, int dv, int j)
 {
     uint32_t u = 0;
     for (int t = 0; t < b; ++t) {
-        int p = j * b + t;
+        int p = code_bit(b, dv, j, t);
         u |= (uint32_t)((row[p / 8] >> (p % 8)) & 1u) << t;
     }
     if (u & (1u << (b - 1))) return (int32_t)u - (int32_t)(1u << b);
     return (int32_t)u;
 }
 
-static void put_code(uint8_t *row, int b, int j, int32_t z)
+static void put_code(uint8_t *row, int b, int dv, int j, int32_t z)
 {
     uint32_t u = (uint32_t)z & ((1u << b) - 1u);
     for (int t = 0; t < b; ++t) {
-        int p = j * b + t;
+        int p = code_bit(b, dv, j, t);
         if ((u >> t) & 1u) row[p / 8] = (uint8_t)(row[p / 8] | (1u << (p % 8)));
         else row[p / 8] = (uint8_t)(row[p / 8] & ~(1u << (p % 8)));
     }
@@ -280,8 +294,8 @@ static void put_col_factor(uint8_t *page, int dk, const uint8_t *bits, int fmt, 
 }
 
 /* exported for the pack/unpack pins */
-int32_t orc_get_code(const uint8_t *row, int b, int j) { return get_code(row, b, j); }
-void orc_put_code(uint8_t *row, int b, int j, int32_t z) { put_code(row, b, j, z); }
+int32_t orc_get_code(const uint8_t *row, int b, int dv, int j) { return get_code(row, b, dv, j); }
+void orc_put_code(uint8_t *row, int b, int dv, int j, int32_t z) { put_code(row, b, dv, j, z); }
 
 /* [steps] step 1, [core]: S^_ij = s_i r_i c_j z_ij, in fp64 (a raw unit: the stored
  * value; a pivot row: z_ij is its binary16 value) */
@@ -297,7 +311,7 @@ static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, con
         }
         double s = (double)get_scale(page, fmt, i);
         for (int j = 0; j < dv; ++j) {
-            double z = bits[i] == 16 ? get_raw(row, 16, j) : (double)get_code(row, bits[i], j);
+            double z = bits[i] == 16 ? get_raw(row, 16, j) : (double)get_code(row, bits[i], dv, j);
             double cj = (double)col_factor(page, dk, bits, fmt, c, j);
             S[(size_t)i * dv + j] = s * (double)r[i] * cj * z;
         }
@@ -318,7 +332,7 @@ static int fit_columns(int dk, int dv, const uint8_t *bits, const float *r, cons
         double num = 0.0, den = 0.0;
         for (int i = 0; i < dk; ++i) {
             const uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
-            double v = (double)get_scale(page, fmt, i) * (double)r[i] * (double)get_code(row, bits[i], j);
+            double v = (double)get_scale(page, fmt, i) * (double)r[i] * (double)get_code(row, bits[i], dv, j);
             double wi = w ? (double)w[i] : 1.0;
             num += wi * wi * v * X[(size_t)i * dv + j];
             den += wi * wi * v * v;
@@ -394,7 +408,7 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
                 z = (int32_t)rz;
             }
             if (quot) quot[(size_t)i * dv + j] = x;
-            put_code(row, bits[i], j, z);
+            put_code(row, bits[i], dv, j, z);
         }
     }
     free(mu);

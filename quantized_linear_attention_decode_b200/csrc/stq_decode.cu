@@ -330,6 +330,9 @@ template <> struct Codec<4> {
 };
 
 template <> struct Codec<6> {
+    // A row is 16 groups of 8 codes; group cg is a 48-bit string (code p at bits
+    // [6p, 6p + 6)) kept as a 32-bit word at byte 4 cg and a 16-bit half at byte
+    // 64 + 2 cg, so both accesses are aligned and no thread straddles another's.
     static constexpr float kMagicOut = 8388640.0f;  // 2^23 + 32: mantissa = u = z + 32 in [1, 63]
     __device__ __forceinline__ static void store(uint8_t *rowg, int cg, const uint32_t b[8])
     {
@@ -337,21 +340,13 @@ template <> struct Codec<6> {
         uint32_t lo = b[0] + (b[1] << 6) + (b[2] << 12) + (b[3] << 18) + (b[4] << 24) + (b[5] << 30);
         lo = (lo - 0x0B000000u) ^ 0x20820820u;
         const uint32_t hi = ((b[5] >> 2) + (b[6] << 4) + (b[7] << 10)) ^ 0x8208u;
-        // 6 bytes at 6 cg: a 4-byte and a 2-byte store, both aligned
-        const uint32_t odd = cg & 1;
-        uint8_t *p = rowg + cg * 6;
-        *reinterpret_cast<uint32_t *>(p + 2 * odd) = odd ? (lo >> 16) | (hi << 16) : lo;
-        *reinterpret_cast<uint16_t *>(p + 4 * (1 - odd)) = static_cast<uint16_t>(odd ? lo : hi);
+        *reinterpret_cast<uint32_t *>(rowg + cg * 4) = lo;
+        *reinterpret_cast<uint16_t *>(rowg + 64 + cg * 2) = static_cast<uint16_t>(hi);
     }
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
-        // 8 codes = 6 bytes at offset 6 cg (2-byte aligned): read the two aligned words around them
-        const uint32_t base = (cg >> 1) * 12 + (cg & 1) * 4;
-        const uint32_t sh = (cg & 1) * 16;
-        const uint32_t w0 = *reinterpret_cast<const uint32_t *>(rowp + base);
-        const uint32_t w1 = *reinterpret_cast<const uint32_t *>(rowp + base + 4);
-        const uint32_t lo = __funnelshift_r(w0, w1, sh);
-        const uint32_t hi = w1 >> sh;
+        const uint32_t lo = *reinterpret_cast<const uint32_t *>(rowp + cg * 4);
+        const uint32_t hi = *reinterpret_cast<const uint16_t *>(rowp + 64 + cg * 2);
         const uint32_t x = lo >> 18;                     // codes 3, 4 at offsets 0, 6
         const uint32_t y = __funnelshift_r(lo, hi, 30);  // codes 5, 6, 7 at offsets 0, 6, 12
         const uint32_t c0 = masked_field<0x3Fu, 0x4B000020u>(lo);     // 2^23 + u

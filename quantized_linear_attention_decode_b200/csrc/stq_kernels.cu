@@ -8,8 +8,11 @@
 //
 // Page layout (one (request, slot, head) tile): 128 fp32 row scales (or 128
 // binary16 scales), then 128 rows of 128 b_i-bit two's complement codes
-// (16 b_i bytes per row, little-endian bit order), padded to 128 bytes.  A raw
-// page is the row-major state itself in binary16 or fp32.
+// (16 b_i bytes per row, little-endian bit order), padded to 128 bytes.  4- and
+// 8-bit code j sits at bits [j b, (j + 1) b) of its row; 6-bit codes go in
+// groups of eight, group g's 48 bits split into a 32-bit word at byte 4 g and a
+// 16-bit half at byte 64 + 2 g.  A raw page is the row-major state itself in
+// binary16 or fp32.
 #include <cstdint>
 
 #include <cuda_fp16.h>
@@ -109,10 +112,11 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
             *reinterpret_cast<uint16_t *>(row + lane * 2) = static_cast<uint16_t>(
                 (code[0] & 15u) | (code[1] & 15u) << 4 | (code[2] & 15u) << 8 | (code[3] & 15u) << 12);
         } else {
+            // lanes 2g, 2g + 1 hold the 8 codes of group g: its 48-bit string is w(2g) | w(2g + 1) << 24
             const uint32_t w = (code[0] & 63u) | (code[1] & 63u) << 6 | (code[2] & 63u) << 12 | (code[3] & 63u) << 18;
-            row[lane * 3 + 0] = static_cast<uint8_t>(w);
-            row[lane * 3 + 1] = static_cast<uint8_t>(w >> 8);
-            row[lane * 3 + 2] = static_cast<uint8_t>(w >> 16);
+            const uint32_t nb = __shfl_xor_sync(0xffffffffu, w, 1);
+            if (lane & 1) *reinterpret_cast<uint16_t *>(row + 64 + (lane >> 1) * 2) = static_cast<uint16_t>(w >> 8);
+            else *reinterpret_cast<uint32_t *>(row + (lane >> 1) * 4) = w | nb << 24;
         }
         if (lane == 0) {
             if (p.scale_bytes == 2) reinterpret_cast<__half *>(page)[i] = s16;
@@ -193,7 +197,9 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
 #pragma unroll
             for (int t = 0; t < 4; ++t) zz[t] = static_cast<int>(w << (28 - 4 * t)) >> 28;
         } else {
-            const uint32_t w = row[lane * 3] | row[lane * 3 + 1] << 8 | row[lane * 3 + 2] << 16;
+            const uint32_t lo = *reinterpret_cast<const uint32_t *>(row + (lane >> 1) * 4);
+            const uint32_t hi = *reinterpret_cast<const uint16_t *>(row + 64 + (lane >> 1) * 2);
+            const uint32_t w = (lane & 1) ? lo >> 24 | hi << 8 : lo & 0xFFFFFFu;
 #pragma unroll
             for (int t = 0; t < 4; ++t) zz[t] = static_cast<int>(w << (26 - 6 * t)) >> 26;
         }

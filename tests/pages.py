@@ -1,8 +1,9 @@
 """Test helpers: read packed pages and compare a GPU step with the oracle.
 
 A vectorised reader of the documented page format (128 fp32 scales, then
-rows of 128 b-bit two's complement codes, little-endian bit order, page
-padded to 128 bytes).  It belongs to neither implementation; the CPU tests
+rows of 128 b-bit two's complement codes, little-endian bit order, 6-bit
+codes in groups of eight split into a word and a half, page padded to 128
+bytes).  It belongs to neither implementation; the CPU tests
 check it against the oracle's bit-by-bit packer.
 """
 from __future__ import annotations
@@ -60,6 +61,10 @@ def decode_page(page: np.ndarray, row_bits, fmt: int = 0) -> tuple[np.ndarray, n
             continue
         nb = 16 * b
         raw = np.stack([page[offs[i]: offs[i] + nb] for i in rows])
+        if b == 6:  # group g: word bytes [4g, 4g+4) then half bytes [64+2g, 66+2g), contiguous again
+            n = len(rows)
+            raw = np.concatenate([raw[:, :64].reshape(n, 16, 4), raw[:, 64:].reshape(n, 16, 2)],
+                                 axis=2).reshape(n, nb)
         bits = np.unpackbits(raw, axis=1, bitorder="little").reshape(len(rows), D, b).astype(np.int64)
         u = (bits << np.arange(b)).sum(axis=2)
         codes[rows] = np.where(u >= (1 << (b - 1)), u - (1 << b), u)

@@ -29,7 +29,7 @@ def _read(page, bits, dv, fmt):
     z = np.zeros((dk, dv), np.int64)
     for i, b in enumerate(bits):
         row = page[offs[i]: offs[i] + dv * int(b) // 8]
-        z[i] = [orc.get_code(row, int(b), j) for j in range(dv)]
+        z[i] = [orc.get_code(row, int(b), j, dv=dv) for j in range(dv)]
     return s, c, z
 
 

@@ -37,7 +37,7 @@ def _codes(page, bits, dv, fmt):
     for i, b in enumerate(bits):
         row = page[offs[i]: offs[i] + dv * int(b) // 8]
         for j in range(dv):
-            z[i, j] = orc.get_code(row, int(b), j)
+            z[i, j] = orc.get_code(row, int(b), j, dv=dv)
     return z
 
 

@@ -28,7 +28,7 @@ def _codes(page, bits, dv):
     for i, b in enumerate(bits):
         row = page[offs[i]: offs[i] + dv * int(b) // 8]
         for j in range(dv):
-            z[i, j] = orc.get_code(row, int(b), j)
+            z[i, j] = orc.get_code(row, int(b), j, dv=dv)
     return z
 
 
@@ -69,10 +69,11 @@ def test_pack_golden_rows():
         codes = [int(x) for x in parts[1].split(",")]
         want = bytes(int(h, 16) for h in parts[2:])
         row = np.zeros(len(want), np.uint8)
+        n = len(codes)
         for j, z in enumerate(codes):
-            orc.put_code(row, b, j, z)
+            orc.put_code(row, b, j, z, dv=n)
         assert row.tobytes() == want, (b, codes, row.tobytes().hex())
-        assert [orc.get_code(row, b, j) for j in range(len(codes))] == codes
+        assert [orc.get_code(row, b, j, dv=n) for j in range(n)] == codes
 
 
 @pytest.mark.parametrize("b", [4, 6, 8])
@@ -199,7 +200,9 @@ def test_quantized_step_continuous_part_matches_explicit_form(kind):
     the explicit-matrix recurrence applied to the reconstructed state."""
     rng = RNG(4)
     for d, bits in ((4, 4), (8, 6), (8, 8)):
-        b = np.full(d, bits, np.uint8) if kind == "gdn" else rng.choice([4, 6, 8], d).astype(np.uint8)
+        # 6-bit rows pack codes in groups of eight, so they need dv % 8 == 0
+        widths = [4, 6, 8] if d % 8 == 0 else [4, 8]
+        b = np.full(d, bits, np.uint8) if kind == "gdn" else rng.choice(widths, d).astype(np.uint8)
         r = np.exp(rng.uniform(-1.4, 1.4, d)).astype(np.float32)
         c = np.exp(rng.uniform(-1.4, 1.4, d)).astype(np.float32)
         page = orc.quantize_unit(b, r, c, rng.standard_normal((d, d)).astype(np.float32))
@@ -371,3 +374,13 @@ def test_synth_is_deterministic_and_shaped():
     wk = synth.make_workload(3, R=2, H=2, T=1)
     rb = wk.row_bits()
     assert rb.shape == (2, 128) and all(sorted(np.bincount(rb[h])[[4, 6, 8]]) == [32, 32, 64] for h in range(2))
+
+
+def test_six_bit_rows_need_whole_groups():
+    """6-bit codes are stored in groups of eight: a unit whose rows hold a
+    number of codes that is not a multiple of 8 has no 6-bit layout."""
+    S = np.ones((8, 4), np.float32)
+    ones = np.ones(8, np.float32)
+    with pytest.raises(ValueError):
+        orc.quantize_unit(np.full(8, 6, np.uint8), ones, np.ones(4, np.float32), S)
+    orc.quantize_unit(np.full(8, 8, np.uint8), ones, np.ones(4, np.float32), S)
