@@ -249,6 +249,34 @@ stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const 
                                   int32_t n, const float *q, const float *k, const float *v,
                                   const float *beta, const float *gate, float *y, void *stream);
 
+/*
+ * stq_decode_step with every per-token buffer in HOST memory: no counterpart
+ * in the paper, for callers that hold their inputs and want y on the host.
+ * Arguments, results and rules are those of stq_decode_step, except that
+ * req_idx, slot_idx, q, k, v, beta, gate and y are host pointers (no
+ * alignment rule).  On `stream`, after the work already queued there, the
+ * library copies the inputs into a device staging buffer that the pool owns,
+ * runs the step (the same kernels, so the results are those of
+ * stq_decode_step bit for bit) and copies y back; y may be read once
+ * `stream` is synchronized.
+ *   - Page-locked host memory (cudaHostAlloc, cudaHostRegister) makes the
+ *     copies asynchronous; pageable memory works, with copies that block the
+ *     host.
+ *   - The inputs must stay unchanged, and y unread, until `stream` has
+ *     passed the step.
+ *   - The first call, and any call with more entries than every earlier
+ *     one, allocates the staging buffer (n * H * 2 KiB, and 512 B more per
+ *     tile for a KDA gate), after waiting on the host for the previous
+ *     host-buffer step of the pool; it is not meant for stream capture.
+ *   - A call on another stream than the pool's previous host-buffer step
+ *     waits for that step (the staging buffer is shared).  Calls on one pool
+ *     from several host threads must be serialized.
+ * Host pointers that are not host memory make a copy fail with STQ_ERR_CUDA.
+ */
+stq_status stq_decode_step_host(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, const float *q, const float *k, const float *v,
+                                const float *beta, const float *gate, float *y, void *stream);
+
 /* Make `stream` wait for the pool's pending split write-back (no-op if none). */
 stq_status stq_pool_join(stq_pool *pool, void *stream);
 

@@ -27,6 +27,11 @@ struct stq_pool {
     // split decode: events behind the last readout and the last write-back
     cudaEvent_t ev_read = nullptr, ev_wb = nullptr;
     mutable bool wb_pending = false;
+    // host-buffer decode: device staging, and an event behind its last use
+    uint8_t *h_stage = nullptr;
+    size_t h_stage_bytes = 0;
+    cudaEvent_t h_done = nullptr;
+    bool h_used = false;
     stq::Tables t{};
     std::vector<uint32_t> head_off, page_bytes;
 };
@@ -415,6 +420,9 @@ stq_status stq_pool_destroy(stq_pool *p)
     if (p->wb_pending) cudaEventSynchronize(p->ev_wb);
     if (p->ev_read) cudaEventDestroy(p->ev_read);
     if (p->ev_wb) cudaEventDestroy(p->ev_wb);
+    if (p->h_used) cudaEventSynchronize(p->h_done);
+    if (p->h_done) cudaEventDestroy(p->h_done);
+    cudaFree(p->h_stage);
     cudaFree(p->d_pages);
     cudaFree(p->d_tables);
     cudaFree(p->d_err);
@@ -645,6 +653,117 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
     stq::DecodeIO wb{req_idx, slot_idx, n, nullptr, k, u, nullptr, gate, nullptr, nullptr};
     e = stq::launch_decode_writeback(view(p), wb, s0);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "write-back launch");
+}
+
+// ---------------------------------------------------------------- decode from host buffers
+//
+// Inputs in, one decode, y out, all on the caller's stream.  Cutting the
+// entries into chunks pipelined over separate copy streams measured slower at
+// 2048 tiles (each cross-stream wait costs more than the overlap it buys) and
+// no faster at 8192, so the step stays on one stream.
+
+}  // extern "C"
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Byte offsets of the staged arrays for n entries (each 256-byte aligned).
+struct HostLayout {
+    size_t req, slot, q, k, v, beta, gate, y, total;
+};
+
+HostLayout host_layout(const stq_pool *p, int32_t n)
+{
+    const size_t vec = (size_t)n * p->H * kD * sizeof(float), per = (size_t)n * p->H * sizeof(float);
+    HostLayout L{};
+    size_t o = 0;
+    L.req = o;  o += align256((size_t)n * sizeof(int32_t));
+    L.slot = o; o += align256((size_t)n * sizeof(int32_t));
+    L.q = o;    o += align256(vec);
+    L.k = o;    o += align256(vec);
+    L.v = o;    o += align256(vec);
+    L.beta = o; o += align256(per);
+    L.gate = o; o += align256(p->kind == STQ_KDA ? vec : per);
+    L.y = o;    o += align256(vec);
+    L.total = o;
+    return L;
+}
+
+// The staging buffer, at least `bytes` long, free for this call's stream to use.
+cudaError_t host_staging(stq_pool *p, size_t bytes, cudaStream_t stream)
+{
+    cudaError_t e = cudaSuccess;
+    if (p->h_done == nullptr) e = cudaEventCreateWithFlags(&p->h_done, cudaEventDisableTiming);
+    if (e != cudaSuccess) return e;
+    if (bytes > p->h_stage_bytes) {
+        // grow: the previous call's copies and launch must be done with the old buffer
+        if (p->h_used) e = cudaEventSynchronize(p->h_done);
+        if (e != cudaSuccess) return e;
+        cudaFree(p->h_stage);
+        p->h_stage = nullptr;
+        p->h_stage_bytes = 0;
+        p->h_used = false;
+        const size_t grown = (bytes + (1u << 20) - 1) & ~static_cast<size_t>((1u << 20) - 1);
+        e = cudaMalloc(&p->h_stage, grown);
+        if (e == cudaSuccess) p->h_stage_bytes = grown;
+        return e;
+    }
+    // the previous call may have run on another stream: wait for it unless it is done
+    if (p->h_used && cudaEventQuery(p->h_done) != cudaSuccess) e = cudaStreamWaitEvent(stream, p->h_done, 0);
+    return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+stq_status stq_decode_step_host(stq_pool *p, const int32_t *req_idx, const int32_t *slot_idx,
+                                int32_t n, const float *q, const float *k, const float *v,
+                                const float *beta, const float *gate, float *y, void *stream)
+{
+    stq_status st = check_launch_args(p, req_idx, slot_idx, n);
+    if (st != STQ_OK) return st;
+    if (n > 0 && (!q || !k || !v || !beta || !gate || !y))
+        return fail(STQ_ERR_ARG, "a q/k/v/beta/gate/y pointer is NULL");
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    const cudaStream_t s0 = (cudaStream_t)stream;
+    const HostLayout L = host_layout(p, n);
+    cudaError_t e = host_staging(p, L.total, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "host-decode staging");
+    e = join_async(p, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    uint8_t *d = p->h_stage;
+    const size_t vec = (size_t)n * p->H * kD * sizeof(float), per = (size_t)n * p->H * sizeof(float);
+    const auto h2d = [&](size_t off, const void *src, size_t bytes) {
+        return cudaMemcpyAsync(d + off, src, bytes, cudaMemcpyHostToDevice, s0);
+    };
+    p->h_used = true;
+    e = h2d(L.req, req_idx, 4 * (size_t)n);
+    if (e == cudaSuccess) e = h2d(L.slot, slot_idx, 4 * (size_t)n);
+    if (e == cudaSuccess) e = h2d(L.q, q, vec);
+    if (e == cudaSuccess) e = h2d(L.k, k, vec);
+    if (e == cudaSuccess) e = h2d(L.v, v, vec);
+    if (e == cudaSuccess) e = h2d(L.beta, beta, per);
+    if (e == cudaSuccess) e = h2d(L.gate, gate, p->kind == STQ_KDA ? vec : per);
+    if (e != cudaSuccess) {
+        cudaEventRecord(p->h_done, s0);
+        return cuda_fail(e, "host-decode input copy");
+    }
+    const stq::DecodeIO io{reinterpret_cast<const int32_t *>(d + L.req), reinterpret_cast<const int32_t *>(d + L.slot),
+                           n, reinterpret_cast<const float *>(d + L.q), reinterpret_cast<const float *>(d + L.k),
+                           reinterpret_cast<const float *>(d + L.v), reinterpret_cast<const float *>(d + L.beta),
+                           reinterpret_cast<const float *>(d + L.gate), reinterpret_cast<float *>(d + L.y), nullptr};
+    e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
+    const cudaError_t eo = e == cudaSuccess ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
+    const cudaError_t er = cudaEventRecord(p->h_done, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (eo != cudaSuccess) return cuda_fail(eo, "host-decode output copy");
+    return er == cudaSuccess ? STQ_OK : cuda_fail(er, "host-decode event");
 }
 
 stq_status stq_pool_join(stq_pool *p, void *stream)

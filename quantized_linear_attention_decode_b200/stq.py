@@ -27,7 +27,7 @@ STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE
 EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
            "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
            "stq_decode_readout", "stq_decode_writeback", "stq_decode_step_split", "stq_pool_join",
-           "stq_decode_step_static", "stq_lifetime_weight", "stq_allocate_bits",
+           "stq_decode_step_static", "stq_decode_step_host", "stq_lifetime_weight", "stq_allocate_bits",
            "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
            "stq_status_str", "stq_last_error")
 
@@ -67,6 +67,7 @@ def load():
         "stq_quantize_state": [P, P, P, I32, P, P],
         "stq_dequantize_state": [P, P, P, I32, P, P],
         "stq_decode_step": [P, P, P, I32, P, P, P, P, P, P, P],
+        "stq_decode_step_host": [P, P, P, I32, P, P, P, P, P, P, P],
         "stq_decode_readout": [P, P, P, I32, P, P, P, P, P, P, P, P],
         "stq_decode_writeback": [P, P, P, I32, P, P, P, P],
         "stq_decode_step_split": [P, P, P, I32, P, P, P, P, P, P, P, P, P],
@@ -228,6 +229,38 @@ def stq_decode_step(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, strea
     _check(load().stq_decode_step(
         pool.handle, r, s, n, _dev(q, f, vec, "q"), _dev(k, f, vec, "k"), _dev(v, f, vec, "v"),
         _dev(beta, f, (n, pool.H), "beta"), _dev(gate, f, gshape, "gate"), _dev(y, f, vec, "y"),
+        _stream(stream)))
+
+
+def _host(t, dtype, shape, name):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be in host memory (pinned for overlapped copies)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+def stq_decode_step_host(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, stream=None) -> None:
+    """stq_decode_step with host (CPU) tensors: the library copies the inputs in,
+    decodes and copies y out, ordered on `stream`; y is valid once `stream` is
+    synchronized.  Keep every tensor referenced (and the inputs unchanged)
+    until then: torch may hand a freed pinned block out again before the
+    library's copy from it has run."""
+    import torch
+    n = int(req_idx.numel())
+    f = torch.float32
+    vec, gshape = _vecs(pool, n)
+    _check(load().stq_decode_step_host(
+        pool.handle, _host(req_idx, torch.int32, (n,), "req_idx"), _host(slot_idx, torch.int32, (n,), "slot_idx"),
+        n, _host(q, f, vec, "q"), _host(k, f, vec, "k"), _host(v, f, vec, "v"),
+        _host(beta, f, (n, pool.H), "beta"), _host(gate, f, gshape, "gate"), _host(y, f, vec, "y"),
         _stream(stream)))
 
 

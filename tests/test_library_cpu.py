@@ -143,6 +143,7 @@ def test_null_arguments_rejected_before_any_cuda_call():
     L = stq.load()
     assert L.stq_pool_create(None, None) == stq.STQ_ERR_ARG
     assert L.stq_decode_step(None, None, None, 0, None, None, None, None, None, None, None) == stq.STQ_ERR_ARG
+    assert L.stq_decode_step_host(None, None, None, 0, None, None, None, None, None, None, None) == stq.STQ_ERR_ARG
     assert L.stq_decode_readout(None, None, None, 0, None, None, None, None, None, None, None,
                                 None) == stq.STQ_ERR_ARG
     assert L.stq_decode_writeback(None, None, None, 0, None, None, None, None) == stq.STQ_ERR_ARG
