@@ -28,6 +28,12 @@
  *     trap is ever raised.
  *   - A call that names the same (request, slot) twice in its index lists
  *     has undefined results (tiles are updated in place, one CTA each).
+ *     With the environment variable STQ_DEBUG_CHECKS=1 set when the pool is
+ *     created, every call that writes pages first runs a check kernel that
+ *     marks each in-range (request, slot) of the call in a bitmap the pool
+ *     owns; a pair seen twice sets the error word, and stq_pool_check then
+ *     returns STQ_ERR_INDEX.  The decode still runs (its results stay
+ *     undefined); the check costs a memset and a launch per call.
  *   - Setting the environment variable STQ_FAULT=alloc makes
  *     stq_pool_create fail with STQ_ERR_OOM, STQ_FAULT=launch makes every
  *     launching call fail with STQ_ERR_CUDA, both before any CUDA call

@@ -24,6 +24,9 @@ struct stq_pool {
     uint8_t *d_pages = nullptr;
     void *d_tables = nullptr;
     uint32_t *d_err = nullptr;
+    // debug checks (STQ_DEBUG_CHECKS=1 at creation): one bit per (request, slot)
+    bool check_dups = false;
+    uint32_t *d_seen = nullptr;
     // split decode: events behind the last readout and the last write-back
     cudaEvent_t ev_read = nullptr, ev_wb = nullptr;
     mutable bool wb_pending = false;
@@ -232,6 +235,13 @@ cudaError_t join_async(const stq_pool *p, cudaStream_t stream)
     return e;
 }
 
+// With debug checks on: flag (request, slot) pairs named twice in one call.
+cudaError_t debug_checks(const stq_pool *p, const int32_t *req, const int32_t *slot, int32_t n, cudaStream_t s)
+{
+    if (!p->check_dups || n == 0) return cudaSuccess;
+    return stq::launch_duplicate_check(req, slot, n, p->R, p->S, p->d_seen, p->d_err, s);
+}
+
 cudaError_t join_host(const stq_pool *p)
 {
     if (!p->wb_pending) return cudaSuccess;
@@ -391,11 +401,16 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     if (e == cudaSuccess) e = cudaMemset(p->d_pages, 0, p->packed_bytes);
     if (e == cudaSuccess) e = cudaMemset(p->d_err, 0, 256);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_tables, img.data(), total, cudaMemcpyHostToDevice);
+    const char *dbg = std::getenv("STQ_DEBUG_CHECKS");
+    p->check_dups = dbg != nullptr && std::strcmp(dbg, "1") == 0;
+    if (e == cudaSuccess && p->check_dups)
+        e = cudaMalloc(&p->d_seen, ((size_t)p->R * p->S + 31) / 32 * sizeof(uint32_t));
     if (e != cudaSuccess) {
         stq_status r = cuda_fail(e, "pool allocation");
         cudaFree(p->d_pages);
         cudaFree(p->d_tables);
         cudaFree(p->d_err);
+        cudaFree(p->d_seen);
         cudaGetLastError();
         delete p;
         return r;
@@ -423,6 +438,7 @@ stq_status stq_pool_destroy(stq_pool *p)
     if (p->h_used) cudaEventSynchronize(p->h_done);
     if (p->h_done) cudaEventDestroy(p->h_done);
     cudaFree(p->h_stage);
+    cudaFree(p->d_seen);
     cudaFree(p->d_pages);
     cudaFree(p->d_tables);
     cudaFree(p->d_err);
@@ -461,6 +477,8 @@ stq_status stq_quantize_state(stq_pool *p, const int32_t *req_idx, const int32_t
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = debug_checks(p, req_idx, slot_idx, n, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "debug checks");
     e = stq::launch_quantize(view(p), req_idx, slot_idx, n, state, (cudaStream_t)stream);
     return e == cudaSuccess ? STQ_OK : cuda_fail(e, "quantize launch");
 }
@@ -495,6 +513,8 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = debug_checks(p, req_idx, slot_idx, n, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "debug checks");
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, nullptr};
     e = p->raw_bits ? stq::launch_decode_raw(view(p), io, (cudaStream_t)stream)
                     : stq::launch_decode(view(p), io, (cudaStream_t)stream);
@@ -541,6 +561,8 @@ stq_status stq_decode_writeback(stq_pool *p, const int32_t *req_idx, const int32
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = debug_checks(p, req_idx, slot_idx, n, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "debug checks");
     // the write-back reads u~ through the v slot; q and beta are not read
     stq::DecodeIO io{req_idx, slot_idx, n, nullptr, k, u_tilde, nullptr, gate, nullptr, nullptr};
     e = stq::launch_decode_writeback(view(p), io, (cudaStream_t)stream);
@@ -567,6 +589,8 @@ stq_status stq_decode_step_split(stq_pool *p, const int32_t *req_idx, const int3
     const cudaStream_t s0 = (cudaStream_t)stream, s1 = (cudaStream_t)side_stream;
     e = join_async(p, s0);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = debug_checks(p, req_idx, slot_idx, n, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "debug checks");
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u_tilde};
     e = stq::launch_decode_readout(view(p), io, s0);
     if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
@@ -645,6 +669,8 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
     const cudaStream_t s0 = (cudaStream_t)stream;
     e = join_async(p, s0);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    e = debug_checks(p, req_idx, slot_idx, n, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "debug checks");
     // the readout fills u~ for every tile of the call before the write-back reads it
     stq::DecodeIO io{req_idx, slot_idx, n, q, k, v, beta, gate, y, u};
     e = stq::launch_decode_readout(view(p), io, s0);
@@ -757,7 +783,8 @@ stq_status stq_decode_step_host(stq_pool *p, const int32_t *req_idx, const int32
                            n, reinterpret_cast<const float *>(d + L.q), reinterpret_cast<const float *>(d + L.k),
                            reinterpret_cast<const float *>(d + L.v), reinterpret_cast<const float *>(d + L.beta),
                            reinterpret_cast<const float *>(d + L.gate), reinterpret_cast<float *>(d + L.y), nullptr};
-    e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
+    e = debug_checks(p, io.req_idx, io.slot_idx, n, s0);
+    if (e == cudaSuccess) e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
     if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
     const cudaError_t eo = e == cudaSuccess ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
     const cudaError_t er = cudaEventRecord(p->h_done, s0);
@@ -817,6 +844,7 @@ stq_status stq_pool_check(stq_pool *p, void *stream)
     if (e != cudaSuccess) return cuda_fail(e, "error word");
     if (word & stq::kErrTimeout) return fail(STQ_ERR_TIMEOUT, "a device-side wait timed out");
     if (word & stq::kErrIndex) return fail(STQ_ERR_INDEX, "request or slot index out of range");
+    if (word & stq::kErrDuplicate) return fail(STQ_ERR_INDEX, "a (request, slot) pair named twice in one call");
     if (word & stq::kErrNonFinite) return fail(STQ_ERR_NONFINITE, "non-finite value in the step");
     return STQ_OK;
 }

@@ -21,6 +21,7 @@ constexpr size_t kStaticScratchFloats = size_t(1) << 20;  // built-in u~ buffer:
 constexpr uint32_t kErrIndex = 1u;
 constexpr uint32_t kErrNonFinite = 2u;
 constexpr uint32_t kErrTimeout = 4u;
+constexpr uint32_t kErrDuplicate = 8u;  // a (request, slot) pair named twice in one call (debug checks)
 
 // Per-head tables, one device allocation:
 //   head_off[H]    byte offset of the head's page inside a slot
@@ -72,6 +73,10 @@ cudaError_t launch_decode_raw(const PoolView &p, const DecodeIO &io, cudaStream_
 cudaError_t launch_decode_pivot_heads(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_readout(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
 cudaError_t launch_decode_writeback(const PoolView &p, const DecodeIO &io, cudaStream_t stream);
+// Marks the call's (request, slot) pairs in `seen` (R * S bits, cleared first on
+// the stream) and sets kErrDuplicate in `err` for a pair named twice.
+cudaError_t launch_duplicate_check(const int32_t *req_idx, const int32_t *slot_idx, int n, int R, int S,
+                                   uint32_t *seen, uint32_t *err, cudaStream_t stream);
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                             int n, const float *state, cudaStream_t stream);
 cudaError_t launch_dequantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,

@@ -273,7 +273,33 @@ __global__ void __launch_bounds__(256) dequantize_raw_kernel(PoolView p, const i
     }
 }
 
+// Debug check: entry e marks bit req * S + slot of `seen` (cleared before the
+// launch); finding it already set means the pair is named twice.  Out-of-range
+// pairs are left to the kernels that follow, which report them.
+__global__ void __launch_bounds__(256) duplicate_kernel(const int32_t *req_idx, const int32_t *slot_idx, int n,
+                                                        int R, int S, uint32_t *seen, uint32_t *err)
+{
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= n) return;
+    const int r = req_idx[e], s = slot_idx[e];
+    if (r < 0 || r >= R || s < 0 || s >= S) return;
+    const uint32_t key = static_cast<uint32_t>(r) * static_cast<uint32_t>(S) + static_cast<uint32_t>(s);
+    const uint32_t bit = 1u << (key & 31u);
+    if (atomicOr(&seen[key >> 5], bit) & bit) atomicOr(err, kErrDuplicate);
+}
+
 }  // namespace
+
+cudaError_t launch_duplicate_check(const int32_t *req_idx, const int32_t *slot_idx, int n, int R, int S,
+                                   uint32_t *seen, uint32_t *err, cudaStream_t stream)
+{
+    const size_t words = (static_cast<size_t>(R) * S + 31) / 32;
+    cudaError_t e = cudaMemsetAsync(seen, 0, words * sizeof(uint32_t), stream);
+    if (e != cudaSuccess) return e;
+    duplicate_kernel<<<(n + 255) / 256, 256, 0, stream>>>(req_idx, slot_idx, n, R, S, seen, err);
+    count_launch();
+    return cudaGetLastError();
+}
 
 cudaError_t launch_quantize(const PoolView &p, const int32_t *req_idx, const int32_t *slot_idx,
                             int n, const float *state, cudaStream_t stream)
