@@ -501,7 +501,7 @@ int orc_step_unit_w(int dk, int dv, const uint8_t *bits, const float *r, const f
         y[j] = acc;
     }
     /* the codes are taken with the unit's current column factors */
-    float *c_now = (float *)malloc(sizeof(float) * (size_t)dv);
+    float *c_now = (float *)calloc((size_t)dv, sizeof(float));
     for (int j = 0; j < dv; ++j) c_now[j] = col_factor(page_in, dk, bits, fmt, c, j);
     memset(page_out, 0, orc_page_bytes_fmt(dk, dv, bits, fmt));
     int st = requantize(dk, dv, bits, r, c_now, w, fmt, P, page_out, quot);
