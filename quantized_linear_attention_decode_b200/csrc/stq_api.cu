@@ -1,6 +1,7 @@
 // stq_api.cu -- host side of the C ABI declared in include/stq.h:
 // pool allocation and tables, argument checking, status and error strings,
 // slot export/import, the device error word, host-side fault injection.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -388,6 +389,21 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
         std::memcpy(blk + 1024, inv_rq, kD * 4);
         std::memcpy(blk + 1536, &img[o_ro + (size_t)h * kD * 2], kD * 2);
         std::memcpy(blk + 1792, &rb[(size_t)h * kD], kD);
+        // the decode kernel's row order (position -> row): KDA rows sorted by width, so
+        // that the two half-warps taking positions 16 w + 2 t and 16 w + 2 t + 1 at step t
+        // of their rows mostly share a width; GDN rows in order
+        uint8_t *perm = blk + 1920;
+        int order[kD];
+        for (int i = 0; i < kD; ++i) order[i] = i;
+        const uint8_t *hb = &rb[(size_t)h * kD];
+        if (p->kind == STQ_KDA) {
+            std::stable_sort(order, order + kD, [hb](int a, int b) { return hb[a] < hb[b]; });
+            for (int w = 0; w < 8; ++w)
+                for (int g = 0; g < 2; ++g)
+                    for (int t = 0; t < 8; ++t) perm[(2 * w + g) * 8 + t] = (uint8_t)order[16 * w + 2 * t + g];
+        } else {
+            for (int i = 0; i < kD; ++i) perm[i] = (uint8_t)i;
+        }
     }
 
     cudaError_t e = cudaGetDevice(&p->device);

@@ -59,7 +59,7 @@ struct __align__(128) Stage {
     float inv_rq[kD];  // 1 / (r_i q_b(i))
     uint16_t row_off[kD];
     uint8_t row_bits[kD];
-    uint8_t pad[kHeadBlock - 3 * 4 * kD - 2 * kD - kD];
+    uint8_t perm[kD];  // KDA: the row taken at each position (rows grouped by width)
     // per-tile vectors, stored from registers by all threads (prefetched two tiles ahead)
     float q[kD], k[kD], v[kD], g[kD];
 };
@@ -67,13 +67,18 @@ static_assert(offsetof(Stage, q) - offsetof(Stage, r) == kHeadBlock, "head block
 static_assert(sizeof(Stage) % 128 == 0, "stage size");
 
 // Per-tile row data, double buffered by tile parity: written while the
-// previous tile finishes, read by both passes of the tile.
+// previous tile finishes, read by both passes of the tile.  Indexed by
+// position: thread (warp w, half g) takes positions 8 (2 w + g) .. + 7.  GDN
+// position i is row i; a KDA head takes its rows in the order of its
+// table's permutation, which groups rows of one width, so that the two
+// halves of a warp mostly unpack and pack rows of the same width together.
 struct __align__(16) RowCoef {
     float4 kl[kD];     // {k_i e_i, k_i e_i, q_i e_i, q_i e_i}
     float h[kD];       // k_i / e_i, or k_i for a dropped row
     float mrq[kD];     // e_i / (r_i q_b(i)) (1 / (r_i q_b) for a dropped row): s'_i = |mrq_i| max_j |w_ij|
     uint16_t off[kD];  // byte offset of row i inside the page
     uint8_t bits[kD];
+    uint8_t row[kD];   // the row at each position
     float fb[kD];      // column fit: (w_i r_i)^2
     uint32_t deg[4];   // bit i: row i's old content is dropped (e_i = 0)
     uint8_t *page;     // the tile's page in global memory
@@ -529,18 +534,19 @@ __device__ __forceinline__ void column_epilogue(Smem &sm, const Stage &S, const 
     if (!isfinite(u) || !isfinite(yj)) atomicOr(&sm.flags, kErrNonFinite);
 }
 
-// Per row (threads 128..255) of the next tile: decayed scale e_i and the
-// coefficients both passes need; warp 4 also forms k.q.
+// Per position (threads 128..255) of the next tile: decayed scale e_i of its
+// row i and the coefficients both passes need; warps 4-7 also form k.q.
 template <int KIND, int SB, int MODE, bool FIT>
 __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, int s)
 {
-    const int r = threadIdx.x - kD;
+    const int pos = threadIdx.x - kD;
     const bool valid = sm.stage_valid[s] != 0;
-    if (r == 0) {
+    if (pos == 0) {
         R.page = sm.stage_page[s];
         R.valid = valid;
     }
     if (!valid) return;
+    const int r = KIND == STQ_KDA ? S.perm[pos] : pos;
     const float sc = SB == 4 ? reinterpret_cast<const float *>(S.page)[r]
                              : __half2float(reinterpret_cast<const __half *>(S.page)[r]);
     const float g = KIND == STQ_GDN ? sm.alpha[s] : S.g[r];
@@ -551,22 +557,23 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     const float ka = kr * e, la = qr * e;
     const float hq = kr * rcp_approx(e);
     const bool dropped = !(e != 0.0f && fabsf(hq) <= 1e30f);
-    R.kl[r] = make_float4(ka, ka, la, la);
-    R.h[r] = dropped ? kr : hq;
-    R.mrq[r] = (dropped ? 1.0f : e) * S.inv_rq[r];
+    R.kl[pos] = make_float4(ka, ka, la, la);
+    R.h[pos] = dropped ? kr : hq;
+    R.mrq[pos] = (dropped ? 1.0f : e) * S.inv_rq[r];
     if (FIT) {
         const float wr = sm.stage_w[s][r] * rr;
-        R.fb[r] = wr * wr;
+        R.fb[pos] = wr * wr;
     }
-    R.off[r] = S.row_off[r];
-    R.bits[r] = S.row_bits[r];
+    R.off[pos] = S.row_off[r];
+    R.bits[pos] = S.row_bits[r];
+    if (KIND == STQ_KDA) R.row[pos] = static_cast<uint8_t>(r);
     const uint32_t bal = __ballot_sync(0xffffffffu, dropped);
-    if ((r & 31) == 0) R.deg[r >> 5] = bal;
+    if ((pos & 31) == 0) R.deg[pos >> 5] = bal;
     if (!isfinite(e)) atomicOr(&sm.flags, kErrNonFinite);
     float a = kr * qr;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if ((r & 31) == 0) R.kqp[r >> 5] = a;
+    if ((pos & 31) == 0) R.kqp[pos >> 5] = a;
 }
 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
@@ -646,7 +653,8 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
         m = fmaxf(m, src[252]);
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
         if (half == 0) {
-            const int i = i0 + ii;
+            const int i = i0 + ii;                 // position
+            const int row = B != 0 ? i : R.row[i];  // its row: the scale slot
             const int b = B != 0 ? B : R.bits[i];
             const float qb = static_cast<float>((1 << (b - 1)) - 1);
             const float mrq = R.mrq[i];
@@ -654,8 +662,8 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
             if (B == 0 && b == 16) {
                 // pivot row: the scale slot keeps 1; mu beyond the binary16 range is reported
                 if (!(fabsf(mrq) * m < 65520.0f)) atomicOr(&sm.flags, kErrNonFinite);
-                if (SB == 4) reinterpret_cast<float *>(page)[i] = 1.0f;
-                else reinterpret_cast<__half *>(page)[i] = __float2half_rn(1.0f);
+                if (SB == 4) reinterpret_cast<float *>(page)[row] = 1.0f;
+                else reinterpret_cast<__half *>(page)[row] = __float2half_rn(1.0f);
             } else if (SB == 4) {
                 if (m >= 1e-30f && m <= 3.0e38f) {
                     inv = copysignf(qb * rcp_approx(m), mrq);
@@ -666,7 +674,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
                 } else if (!(m == 0.0f)) {
                     atomicOr(&sm.flags, kErrNonFinite);
                 }
-                reinterpret_cast<float *>(page)[i] = snew;
+                reinterpret_cast<float *>(page)[row] = snew;
                 if (FIT) {
                     // A = w^2 r e~ s' = (w r)^2 q_b mrq s', since mrq = e~ / (r q_b)
                     sm.rowA[i] = ((R.fb[i] * qb) * mrq) * snew;
@@ -683,7 +691,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
                 // for a normal binary16 scale s / s16 <= 1 + 2^-11, so |w inv| <= q_b (1 + 2^-11)
                 // rounds to at most q_b (q_b <= 127); only a subnormal s16 can round further down
                 clip = sf < s && sf < 6.103515625e-05f;
-                reinterpret_cast<__half *>(page)[i] = s16;
+                reinterpret_cast<__half *>(page)[row] = s16;
                 if (FIT) {
                     const float sv = sf <= 65504.0f ? sf : 0.0f;
                     sm.rowA[i] = ((R.fb[i] * qb) * mrq) * sv;

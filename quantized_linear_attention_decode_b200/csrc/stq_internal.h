@@ -30,9 +30,9 @@ constexpr uint32_t kErrDuplicate = 8u;  // a (request, slot) pair named twice in
 //   row_bits[H][128]
 //   r[H][128], c[H][128]
 //   w[H][128]       row weights of the column fit
-//   block[H][kHeadBlock]: r, c, 1 / (r q_b), row_off, row_bits of one head
+//   block[H][kHeadBlock]: r, c, 1 / (r q_b), row_off, row_bits, decode row order of one head
 //                  side by side, so that the decode kernel fetches them with one copy
-constexpr int kHeadBlock = 2048;  // 512 (r) + 512 (c) + 512 (1 / (r q_b)) + 256 (row_off) + 128 (row_bits), padded
+constexpr int kHeadBlock = 2048;  // 512 (r) + 512 (c) + 512 (1 / (r q_b)) + 256 (row_off) + 128 (row_bits) + 128 (row order)
 constexpr int kFitBytes = 4 * kD;  // a fitted page's own column factors (fp32), after the scales
 struct Tables {
     const uint32_t *head_off;
