@@ -79,6 +79,7 @@ struct __align__(16) RowCoef {
     uint16_t off[kD];  // byte offset of row i inside the page
     uint8_t bits[kD];
     uint8_t row[kD];   // the row at each position
+    uint8_t wbits[8];  // KDA: the width all 16 positions of pass warp w share, else 0
     float fb[kD];      // column fit: (w_i r_i)^2
     uint32_t deg[4];   // bit i: row i's old content is dropped (e_i = 0)
     uint8_t *page;     // the tile's page in global memory
@@ -426,9 +427,10 @@ __device__ __forceinline__ float magic_out(int b)
 // updated row values w.
 //
 // Pass 1: unpack the old codes, accumulate the two column sums and leave
-// per-warp partials in red.  B = 4, 6, 8: every row has B
-// bits (GDN); B = 0: per-row widths (KDA).
-template <int B, int SB, bool FIT, bool ACC = true>
+// per-warp partials in red.  B = 4, 6, 8: every row has B bits, at
+// 16 B i (GDN) or, with PR, at the row table's offsets (a KDA warp whose
+// rows share one width); B = 0: per-row widths (KDA).
+template <int B, int SB, bool FIT, bool ACC = true, bool PR = false>
 __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -441,7 +443,8 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
-        if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
+        if (B != 0 && PR) Codec<B == 0 ? 8 : B>::unpack(S.page + R.off[i], cg, z[ii]);
+        else if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
         else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
         if constexpr (ACC) {
             const float4 kl = R.kl[i];
@@ -566,7 +569,13 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
     }
     R.off[pos] = S.row_off[r];
     R.bits[pos] = S.row_bits[r];
-    if (KIND == STQ_KDA) R.row[pos] = static_cast<uint8_t>(r);
+    if (KIND == STQ_KDA) {
+        R.row[pos] = static_cast<uint8_t>(r);
+        // pass warp pos / 16 takes positions [16 (pos / 16), + 16): one width for all, or 0
+        const uint32_t same = __match_any_sync(0xffffffffu, static_cast<uint32_t>(S.row_bits[r]));
+        const uint32_t half = 0xFFFFu << (pos & 16);
+        if ((pos & 15) == 0) R.wbits[pos >> 4] = (same & half) == half ? S.row_bits[r] : 0;
+    }
     const uint32_t bal = __ballot_sync(0xffffffffu, dropped);
     if ((pos & 31) == 0) R.deg[pos >> 5] = bal;
     if (!isfinite(e)) atomicOr(&sm.flags, kErrNonFinite);
@@ -579,7 +588,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
 // groups of the half-warp through shared memory), new scale, requantise,
 // store codes and scales to the page in global memory.
-template <int B, int SB, bool FIT>
+template <int B, int SB, bool FIT, bool PR = false>
 __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -654,7 +663,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
         if (half == 0) {
             const int i = i0 + ii;                 // position
-            const int row = B != 0 ? i : R.row[i];  // its row: the scale slot
+            const int row = B != 0 && !PR ? i : R.row[i];  // its row: the scale slot
             const int b = B != 0 ? B : R.bits[i];
             const float qb = static_cast<float>((1 << (b - 1)) - 1);
             const float mrq = R.mrq[i];
@@ -751,7 +760,8 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
                 fden[p] = ffma2(make_float2(Bc, Bc), fmul2(zq, zq), fden[p]);
             }
         }
-        if (B != 0) Codec<B == 0 ? 8 : B>::store(rows + 16 * B * i, cg, bits);
+        if (B != 0 && PR) Codec<B == 0 ? 8 : B>::store(page + R.off[i], cg, bits);
+        else if (B != 0) Codec<B == 0 ? 8 : B>::store(rows + 16 * B * i, cg, bits);
         else store_any(b, page + R.off[i], cg, bits);
     }
     if (FIT) {
@@ -952,7 +962,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         float2 z[8][4];
         constexpr bool kAcc = MODE != kWriteback;
         if (valid) {
-            if (KIND == STQ_KDA) pass1<0, SB, FIT, kAcc>(sm, S, R, z);  // per-row widths (and KDA pivot rows)
+            if constexpr (KIND == STQ_KDA) {
+                // per-row widths (and KDA pivot rows), or the one width of this warp's rows
+                const int wb = R.wbits[tid >> 5];
+                if (wb == 6) pass1<6, SB, FIT, kAcc, true>(sm, S, R, z);
+                else if (wb == 8) pass1<8, SB, FIT, kAcc, true>(sm, S, R, z);
+                else if (wb == 4) pass1<4, SB, FIT, kAcc, true>(sm, S, R, z);
+                else pass1<0, SB, FIT, kAcc>(sm, S, R, z);
+            }
             else if (b == 8) pass1<8, SB, FIT, kAcc>(sm, S, R, z);
             else if (b == 6) pass1<6, SB, FIT, kAcc>(sm, S, R, z);
             else pass1<4, SB, FIT, kAcc>(sm, S, R, z);
@@ -986,7 +1003,13 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         timed_out = __syncthreads_or(tout) != 0;
         if (valid && MODE != kReadout) {
-            if (KIND == STQ_KDA) pass2<0, SB, FIT>(sm, R, z);
+            if constexpr (KIND == STQ_KDA) {
+                const int wb = R.wbits[tid >> 5];
+                if (wb == 6) pass2<6, SB, FIT, true>(sm, R, z);
+                else if (wb == 8) pass2<8, SB, FIT, true>(sm, R, z);
+                else if (wb == 4) pass2<4, SB, FIT, true>(sm, R, z);
+                else pass2<0, SB, FIT>(sm, R, z);
+            }
             else if (b == 8) pass2<8, SB, FIT>(sm, R, z);
             else if (b == 6) pass2<6, SB, FIT>(sm, R, z);
             else pass2<4, SB, FIT>(sm, R, z);
