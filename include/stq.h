@@ -134,7 +134,8 @@ typedef struct {
  * and every step rounds X once (to nearest even) into it.
  */
 
-/* Allocate a pool (device memory, all states zero) for the current device. */
+/* Allocate a pool (device memory, all states zero) for the current device.
+ * With STQ_FIT_COLUMNS every page's column factors start as col_factor. */
 stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out);
 stq_status stq_pool_destroy(stq_pool *pool);
 

@@ -417,6 +417,20 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     if (e == cudaSuccess) e = cudaMemset(p->d_pages, 0, p->packed_bytes);
     if (e == cudaSuccess) e = cudaMemset(p->d_err, 0, 256);
     if (e == cudaSuccess) e = cudaMemcpy(p->d_tables, img.data(), total, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && p->fit) {
+        // a zero state still carries column factors: every page starts with the pool's
+        // col_factor (the factors the first step takes its codes with, and refits)
+        std::vector<uint8_t> slot(p->slot_bytes, 0);
+        const float *fcs = reinterpret_cast<const float *>(&img[o_c]);
+        for (int h = 0; h < H; ++h)
+            std::memcpy(&slot[p->head_off[h] + (size_t)p->scale_bytes * kD], fcs + (size_t)h * kD, kD * 4);
+        const size_t units = (size_t)p->R * p->S;
+        e = cudaMemcpy(p->d_pages, slot.data(), p->slot_bytes, cudaMemcpyHostToDevice);
+        for (size_t done = 1; e == cudaSuccess && done < units; done *= 2) {
+            const size_t n = std::min(done, units - done);
+            e = cudaMemcpy(p->d_pages + done * p->slot_bytes, p->d_pages, n * p->slot_bytes, cudaMemcpyDeviceToDevice);
+        }
+    }
     const char *dbg = std::getenv("STQ_DEBUG_CHECKS");
     p->check_dups = dbg != nullptr && std::strcmp(dbg, "1") == 0;
     if (e == cudaSuccess && p->check_dups)

@@ -139,3 +139,30 @@ def test_fit_split_bit_identical_to_fused():
             assert stq.stq_export_slot(a, r, 0).tobytes() == stq.stq_export_slot(b, r, 0).tobytes()
     a.close()
     b.close()
+
+
+def test_fit_kda_f16_scales_split():
+    """KDA rows (warps of one width take the width-specialised passes) with binary16
+    scales and fitted factors, through the split step's readout and write-back."""
+    wl = dataclasses.replace(synth.make_workload(3, R=2, H=4), init="outlier")
+    _teacher_forced(wl, _weights(wl, 5), steps=6, f16=True, split=True)
+
+
+def test_fit_zero_start_pages_carry_initial_factors():
+    """A fitted pool that was never quantized holds zero states whose pages carry
+    the pool's col_factor; decoding from there matches the oracle (KDA, binary16 scales)."""
+    wl = synth.make_workload(3, R=2, H=4)
+    assert wl.initial_state() is None
+    wl = dataclasses.replace(wl, col_factor=synth.log_uniform(synth.stream_key(0, 3, 99), wl.H * 128, 0.5, 2.0)
+                             .astype(np.float32))
+    w = _weights(wl, 6)
+    pool, _, _ = _pool(wl, w, True)
+    rb = wl.row_bits()
+    fmt = FITC | 1
+    c = wl.col_factor.reshape(wl.H, 128)
+    for a in range(wl.R):
+        for h, page in enumerate(split_slot(stq.stq_export_slot(pool, a, 0), rb, fmt)):
+            np.testing.assert_array_equal(col_factors(page, rb[h], fmt), c[h])
+            assert not page[:256].any() and not page[256 + 512:].any()
+    pool.close()
+    _teacher_forced(wl, w, steps=4, f16=True)

@@ -22,9 +22,9 @@ def _host(a, pinned):
     return t.pin_memory() if pinned else t.clone()
 
 
-def _pool(wl, unit_bits=None):
+def _pool(wl, unit_bits=None, flags=0):
     ub = wl.unit_bits if unit_bits is None else unit_bits
-    pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, ub, wl.row_factor, wl.col_factor)
+    pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, ub, wl.row_factor, wl.col_factor, flags=flags)
     req = _cuda(np.arange(wl.R, dtype=np.int32))
     slot = _cuda(wl.slot_of_request.astype(np.int32))
     S0 = wl.initial_state()
@@ -38,10 +38,10 @@ def _slots(pool, wl):
     return [stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])) for a in range(wl.R)]
 
 
-def _run_twins(wl, steps, *, pinned=True, entries=None, unit_bits=None, stream=None):
+def _run_twins(wl, steps, *, pinned=True, entries=None, unit_bits=None, stream=None, flags=0):
     """Advance twin pools `steps` tokens, one through device buffers and one
     through host buffers; return both pools' y and slots."""
-    ref, got = _pool(wl, unit_bits), _pool(wl, unit_bits)
+    ref, got = _pool(wl, unit_bits, flags), _pool(wl, unit_bits, flags)
     for t in range(steps):
         sel = np.arange(wl.R) if entries is None else np.asarray(entries[t])
         n = len(sel)
@@ -147,3 +147,11 @@ def test_host_decode_alternating_streams():
     _same_slots(_slots(ref, wl), _slots(got, wl))
     ref.close()
     got.close()
+
+
+@pytest.mark.parametrize("config, flags", [(3, stq.STQ_SCALE_F16), (2, stq.STQ_FIT_COLUMNS),
+                                           (3, stq.STQ_FIT_COLUMNS | stq.STQ_SCALE_F16)])
+def test_host_decode_scale_and_fit_formats(config, flags):
+    """Binary16 scales and fitted column factors go through the host-buffer step unchanged."""
+    wl = synth.make_workload(config, R=12, H=8)
+    _same_slots(*_run_twins(wl, 3, flags=flags))
