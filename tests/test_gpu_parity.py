@@ -102,6 +102,52 @@ def _teacher_forced(wl, steps, units=None, check_steps=None, split=False):
     return cmp
 
 
+def _free_running(wl, steps):
+    """Both sides advance their own chains from the same quantized start (the GPU's
+    quantizer is bit-exact with the oracle's).  A unit is compared at every step
+    until its first logged near-tie: after one, the two chains may differ by an
+    LSB that the following steps carry forward.  Returns the comparison record
+    and the number of unit-steps compared."""
+    pool = _pool(wl)
+    req, slot = _init(wl, pool)
+    rb = wl.row_bits()
+    own = {}
+    for a in range(wl.R):
+        for h, page in enumerate(split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb)):
+            own[(a, h)] = page.copy()
+    live = set(own)
+    cmp = Compare()
+    compared = 0
+    for t in range(steps):
+        inp, y = _step(wl, pool, req, slot, t)
+        for a in range(wl.R):
+            after = split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb)
+            for h in range(wl.H):
+                page_ref, y_ref, quot, st = _oracle_unit(wl, rb, own[(a, h)], inp, a, h)
+                assert st == orc.OK
+                own[(a, h)] = page_ref
+                if (a, h) not in live:
+                    continue
+                where = f"(free-running t={t}, req={a}, head={h})"
+                ties = len(cmp.ties)
+                cmp.y(y[a, h], y_ref, where)
+                cmp.page(after[h], page_ref, quot, rb[h], where)
+                compared += 1
+                if len(cmp.ties) > ties:
+                    live.discard((a, h))
+    cmp.finish()
+    pool.close()
+    return cmp, compared
+
+
+@pytest.mark.parametrize("config, R, H, steps", [(2, 2, 8, 12), (3, 2, 4, 12)])
+def test_decode_free_running(config, R, H, steps):
+    """GDN mixed with outlier start, and KDA from zero: no teacher forcing."""
+    wl = synth.make_workload(config, R=R, H=H)
+    cmp, compared = _free_running(wl, steps)
+    assert compared >= R * H * steps // 2, (compared, len(cmp.ties))
+
+
 # ---------------------------------------------------------------- quantize / dequantize
 
 
