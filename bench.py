@@ -345,7 +345,7 @@ def run_ours(args, rank: int, world: int):
     torch.cuda.synchronize()
     n0 = stq.stq_launch_count()
     sampler = ClockSampler(dev)
-    with sampler:
+    with sampler, torch.cuda.nvtx.range("bench: timed decode steps"):
         for i in range(args.steps):
             flush.zero_()
             starts[i].record(stream)
@@ -407,13 +407,16 @@ def run_ours(args, rank: int, world: int):
 
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
-        sweep = pool_sweep(stq, flush, stream, peak)
+        with torch.cuda.nvtx.range("bench: pool sweep"):
+            sweep = pool_sweep(stq, flush, stream, peak)
     loop = None
     if rank == 0 and world == 1 and not args.no_layer_loop:
-        loop = layer_loop(stq, flush)
+        with torch.cuda.nvtx.range("bench: layer loop"):
+            loop = layer_loop(stq, flush)
     drift_log = None
     if rank == 0 and world == 1 and not args.no_drift:
-        drift_log = drift(stq)
+        with torch.cuda.nvtx.range("bench: drift"):
+            drift_log = drift(stq)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -12,6 +12,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "stq_internal.h"
 
 struct stq_pool {
@@ -196,6 +198,15 @@ stq::PoolView view(stq_pool *p)
     v.err = p->d_err;
     return v;
 }
+
+// An NVTX range over a launching call (a no-op unless a profiler is attached),
+// so that profiles attribute device work to the entry point that queued it.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Makes the pool's device current for the duration of a call.
 struct DeviceGuard {
@@ -504,6 +515,7 @@ stq_status stq_quantize_state(stq_pool *p, const int32_t *req_idx, const int32_t
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_quantize_state");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
@@ -524,6 +536,7 @@ stq_status stq_dequantize_state(stq_pool *p, const int32_t *req_idx, const int32
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_dequantize_state");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
@@ -540,6 +553,7 @@ stq_status stq_decode_step(stq_pool *p, const int32_t *req_idx, const int32_t *s
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_step");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
@@ -564,6 +578,7 @@ stq_status stq_decode_readout(stq_pool *p, const int32_t *req_idx, const int32_t
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_readout");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
@@ -588,6 +603,7 @@ stq_status stq_decode_writeback(stq_pool *p, const int32_t *req_idx, const int32
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_writeback");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = join_async(p, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
@@ -611,6 +627,7 @@ stq_status stq_decode_step_split(stq_pool *p, const int32_t *req_idx, const int3
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_step_split");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     cudaError_t e = cudaSuccess;
     if (p->ev_read == nullptr) e = cudaEventCreateWithFlags(&p->ev_read, cudaEventDisableTiming);
@@ -692,6 +709,7 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_step_static");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     float *u = nullptr;
     cudaError_t e = static_u_tilde(p->device, &u);
@@ -785,6 +803,7 @@ stq_status stq_decode_step_host(stq_pool *p, const int32_t *req_idx, const int32
     if (n == 0) return STQ_OK;
     if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
     DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_step_host");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
     const cudaStream_t s0 = (cudaStream_t)stream;
     const HostLayout L = host_layout(p, n);
