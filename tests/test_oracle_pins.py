@@ -384,3 +384,55 @@ def test_six_bit_rows_need_whole_groups():
     with pytest.raises(ValueError):
         orc.quantize_unit(np.full(8, 6, np.uint8), ones, np.ones(4, np.float32), S)
     orc.quantize_unit(np.full(8, 8, np.uint8), ones, np.ones(4, np.float32), S)
+
+
+# ---------------------------------------------------------------- the multi-unit driver
+
+
+@pytest.mark.parametrize("nthreads", [1, 4])
+def test_step_many_matches_unit_by_unit(nthreads):
+    """The OpenMP driver that the CPU baseline times advances each unit
+    exactly as a single-unit step does: per-head tables picked by head index,
+    pages read and written at the given (shuffled, distinct) offsets, per-unit
+    vectors and per-row gates.  Heads mix GDN-like uniform widths with
+    KDA-like per-row widths, so a wrong head index, table stride or page offset
+    changes some unit's page or readout."""
+    rng = RNG(11)
+    H, n = 5, 12
+    bits = np.stack([np.full(128, 8, np.uint8), np.full(128, 4, np.uint8), np.full(128, 6, np.uint8),
+                     rng.permutation(np.repeat(np.array([4, 6, 8], np.uint8), [32, 64, 32])),
+                     rng.permutation(np.repeat(np.array([4, 8], np.uint8), [64, 64]))])
+    r = np.exp(rng.uniform(-1, 1, (H, 128))).astype(np.float32)
+    c = np.exp(rng.uniform(-1, 1, (H, 128))).astype(np.float32)
+    head = rng.integers(0, H, n).astype(np.int32)
+    head[:H] = np.arange(H)  # every head at least once
+    sizes = np.array([orc.page_bytes(bits[h]) for h in head])
+    # input pages packed in unit order; output pages in a shuffled order with gaps
+    off_in = np.concatenate([[0], np.cumsum(sizes)[:-1]]).astype(np.int64)
+    order = rng.permutation(n)
+    off_out = np.zeros(n, np.int64)
+    o = 64
+    for u in order:
+        off_out[u] = o
+        o += sizes[u] + 128
+    pages_in = np.zeros(int(sizes.sum()), np.uint8)
+    for u in range(n):
+        S = rng.standard_normal((128, 128)).astype(np.float32)
+        pages_in[off_in[u]: off_in[u] + sizes[u]] = orc.quantize_unit(bits[head[u]], r[head[u]], c[head[u]], S)
+    q = np.stack([_unit(128, rng) for _ in range(n)])
+    k = np.stack([_unit(128, rng) for _ in range(n)])
+    v = rng.standard_normal((n, 128)).astype(np.float32)
+    beta = rng.uniform(0, 1, n).astype(np.float32)
+    g = rng.uniform(0.8, 1.0, (n, 128)).astype(np.float32)
+    out, y, bad = orc.step_many(head, bits, r, c, pages_in, off_in, off_out, o, q, k, v, beta, g, nthreads)
+    assert bad == 0
+    covered = np.zeros(o, bool)
+    for u in range(n):
+        h = head[u]
+        ref, yref, _, st = orc.step_unit(bits[h], r[h], c[h], pages_in[off_in[u]: off_in[u] + sizes[u]],
+                                         q[u], k[u], v[u], beta[u], g[u])
+        assert st == orc.OK
+        np.testing.assert_array_equal(out[off_out[u]: off_out[u] + sizes[u]], ref, err_msg=f"unit {u} page")
+        np.testing.assert_array_equal(y[u], yref, err_msg=f"unit {u} readout")
+        covered[off_out[u]: off_out[u] + sizes[u]] = True
+    assert not out[~covered].any(), "bytes written outside the units' output pages"
