@@ -58,8 +58,12 @@
  *     factors; a column whose codes are all zero keeps its factor.  With one
  *     absmax scale per row, r_i cancels from codes and reconstruction alike,
  *     so the row factor's online formula r_i = m_i^(1/2) w_i^(-1/2) changes
- *     nothing here and is not evaluated.  Pivot rows are not combined with
- *     the fit;
+ *     nothing here and is not evaluated;
+ *   - pivot rows in a fitted unit ([core]: c_j is fitted "across non-pivot
+ *     rows"): the fit sums run over the non-pivot rows only, and a pivot row
+ *     stores mu_ij = fl32(X_ij / r_i) without the column factor (its value
+ *     must not move when the factors are refitted), reconstructing as
+ *     s_i r_i mu_ij with s_i = 1;
  *   - the continuous part (reconstruction, decay, retrieval, write,
  *     readout) is computed in fp64; the quantisation decision is taken in
  *     fp32 on the fp32-rounded value mu_ij = fl32(X_ij / (r_i c_j)), with
@@ -106,8 +110,7 @@ static size_t row_bytes(int dv, int b) { return (size_t)dv * (size_t)b / 8u; }
 
 static int fmt_ok(int fmt)
 {
-    if (fmt < 0 || (fmt & ~(ORC_FMT_F16 | ORC_FMT_PIVOT | ORC_FMT_FITC)) != 0) return 0;
-    return !((fmt & ORC_FMT_PIVOT) && (fmt & ORC_FMT_FITC));
+    return fmt >= 0 && (fmt & ~(ORC_FMT_F16 | ORC_FMT_PIVOT | ORC_FMT_FITC)) == 0;
 }
 
 /* 16 or 32 for a raw unit (its first row decides; bits_ok checks the rest), else 0 */
@@ -310,9 +313,10 @@ static void reconstruct(int dk, int dv, const uint8_t *bits, const float *r, con
             continue;
         }
         double s = (double)get_scale(page, fmt, i);
+        int pivot_fit = bits[i] == 16 && (fmt & ORC_FMT_FITC);
         for (int j = 0; j < dv; ++j) {
             double z = bits[i] == 16 ? get_raw(row, 16, j) : (double)get_code(row, bits[i], dv, j);
-            double cj = (double)col_factor(page, dk, bits, fmt, c, j);
+            double cj = pivot_fit ? 1.0 : (double)col_factor(page, dk, bits, fmt, c, j);
             S[(size_t)i * dv + j] = s * (double)r[i] * cj * z;
         }
     }
@@ -331,6 +335,7 @@ static int fit_columns(int dk, int dv, const uint8_t *bits, const float *r, cons
     for (int j = 0; j < dv; ++j) {
         double num = 0.0, den = 0.0;
         for (int i = 0; i < dk; ++i) {
+            if (bits[i] == 16) continue; /* pivot rows are not part of the fit */
             const uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
             double v = (double)get_scale(page, fmt, i) * (double)r[i] * (double)get_code(row, bits[i], dv, j);
             double wi = w ? (double)w[i] : 1.0;
@@ -373,11 +378,12 @@ static int requantize(int dk, int dv, const uint8_t *bits, const float *r, const
     float *mu = (float *)malloc(sizeof(float) * (size_t)dv);
     for (int i = 0; i < dk; ++i) {
         if (bits[i] == 16) {
-            /* pivot row: scale slot 1, mu rounded once to binary16; quot receives mu */
+            /* pivot row: scale slot 1, mu rounded once to binary16 (in a fitted unit without
+             * the column factor); quot receives mu */
             uint8_t *row = page + row_offset(dk, dv, bits, fmt, i);
             put_scale(page, fmt, i, 1.0f);
             for (int j = 0; j < dv; ++j) {
-                double rc = (double)r[i] * (double)c[j];
+                double rc = (fmt & ORC_FMT_FITC) ? (double)r[i] : (double)r[i] * (double)c[j];
                 float m = (float)(X[(size_t)i * dv + j] / rc);
                 double st = put_raw(row, 16, j, (double)m);
                 if (!isfinite(st)) status = ORC_NONFINITE;
