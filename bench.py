@@ -88,10 +88,15 @@ def recorded_traffic(config: int):
     return e.get("dram_bytes_per_launch")
 
 
-def workload_info(wl):
-    rb = wl.row_bits().astype(np.int64)
-    per_head = [synth.algorithmic_bytes_per_head_step(wl.kind, int(rb[h].sum())) for h in range(wl.H)]
-    tables = wl.H * (2 * 128 * 4)  # r and c read once per head per launch
+def workload_info(wl, unit_bits=None, scale_bytes: int = 4):
+    """(algorithmic HBM bytes of one launch over the whole workload, mean
+    bits per state value); `unit_bits` replaces the workload's widths (a raw
+    fp16 / fp32 pool, scale_bytes 0)."""
+    ub = wl.unit_bits if unit_bits is None else np.asarray(unit_bits)
+    rb = (np.repeat(ub.reshape(wl.H, 1), 128, axis=1) if wl.kind == synth.GDN else ub.reshape(wl.H, 128))
+    rb = rb.astype(np.int64)
+    per_head = [synth.algorithmic_bytes_per_head_step(wl.kind, int(rb[h].sum()), scale_bytes) for h in range(wl.H)]
+    tables = wl.H * (2 * 128 * 4) if scale_bytes else 0  # r and c read once per head per launch
     bytes_per_launch = wl.R * sum(per_head) + tables
     return bytes_per_launch, float(rb.mean())
 
@@ -368,23 +373,29 @@ def run_ours(args, rank: int, world: int):
     achieved = bytes_per_launch / kernel_s / 1e9
     traffic = recorded_traffic(args.config)
 
-    # ---- end to end through the public API: pinned host inputs in, y out, through
-    # stq_decode_step_host (its copies and the decode are in the timed interval)
+    # ---- end to end through the public API: one pinned host block of inputs in,
+    # y out, through stq_decode_step_host_block (its two copies and the decode are
+    # in the timed interval)
     e2e = None
     if args.e2e_steps > 0:
-        host = []
+        n = wl.R
+        offs, nbytes = stq.stq_host_block_layout(pool, n)
+        blocks = []
         for t in range(min(ntok, 16)):
-            host.append({k: v.cpu().pin_memory() for k, v in toks[t].items()})
-        req_h = req.cpu().pin_memory()
-        slot_h = slot.cpu().pin_memory()
+            blk = torch.zeros(nbytes, dtype=torch.uint8).pin_memory()
+            raw = blk.numpy()
+            parts = [req.cpu().numpy(), slot.cpu().numpy()] + [toks[t][k].cpu().numpy()
+                                                               for k in ("q", "k", "v", "beta", "gate")]
+            for o, a in zip(offs, parts):
+                b = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+                raw[o: o + b.size] = b
+            blocks.append(blk)
         y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        h2d = req_h.numel() * 4 + slot_h.numel() * 4 + sum(v.numel() * v.element_size() for v in host[0].values())
+        h2d = nbytes
         d2h = y.numel() * y.element_size()
 
         def host_step(i):
-            x = host[i % len(host)]
-            stq.stq_decode_step_host(pool, req_h, slot_h, x["q"], x["k"], x["v"], x["beta"], x["gate"],
-                                     y_host, stream)
+            stq.stq_decode_step_host_block(pool, n, blocks[i % len(blocks)], y_host, stream)
 
         for i in range(args.warmup):
             host_step(i)
@@ -400,10 +411,16 @@ def run_ours(args, rank: int, world: int):
             e_e[i].record(stream)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(float(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))), dist, "cuda")
+        stq.stq_pool_check(pool, stream)
+        # the box's pinned copy rates for the same byte counts (plain copies, no decode)
+        h2d_s, d2h_s = copy_rates(torch, blocks[0], y_host, stream)
+        step_s = e_ms * 1e-3 / args.e2e_steps
         e2e = {"value": world * units * args.e2e_steps / (e_ms * 1e-3), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": "stq_decode_step_host (pinned host buffers)"}
-        stq.stq_pool_check(pool, stream)
+               "api": "stq_decode_step_host_block (one pinned host block in, y out)",
+               "ms_per_step": step_s * 1e3,
+               "pinned_h2d_gbs": h2d / h2d_s / 1e9, "pinned_d2h_gbs": d2h / d2h_s / 1e9,
+               "copies_plus_kernel_ms": (h2d_s + d2h_s + kernel_s) * 1e3}
 
     sweep = None
     if rank == 0 and world == 1 and not args.no_sweep:
@@ -454,37 +471,73 @@ def run_ours(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
+def copy_rates(torch, host_in, host_out, stream, reps: int = 20):
+    """Median seconds of one pinned host-to-device copy of `host_in` and one
+    device-to-host copy into `host_out` (plain copies on `stream`)."""
+    dev_in = torch.empty(host_in.shape, dtype=host_in.dtype, device="cuda")
+    dev_out = torch.empty(host_out.shape, dtype=host_out.dtype, device="cuda")
+    out = []
+    for src, dst in ((host_in, dev_in), (dev_out, host_out)):
+        ts = []
+        for i in range(reps + 3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            dst.copy_(src, non_blocking=True)
+            b.record(stream)
+            if i >= 3:
+                ts.append((a, b))
+        torch.cuda.synchronize()
+        out.append(statistics.median(a.elapsed_time(b) for a, b in ts) * 1e-3)
+    return out[0], out[1]
+
+
 def pool_sweep(stq, flush, stream, peak, reps: int = 20):
     """Serving-pool sweep: R requests x 5 slots x 768 heads (48 layers x 16
-    heads), mixed 6-bit GDN, one token per launch over all heads; median
-    kernel time over `reps` launches with the L2 flushed before each."""
+    heads), one token per launch over all heads; median kernel time over
+    `reps` launches with the L2 flushed before each.  Each R runs the mixed
+    6-bit GDN pool, and the same shape with an unquantized fp32 state (the
+    page's FP32 control) and a binary16 state; fp32_over_quant is the
+    state-update speedup of the quantized pool over the fp32 one."""
     import torch
     out = []
     for R in (16, 32, 64, 128, 256):
         wl = synth.make_workload(4, R=R)
-        pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
         req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
         slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
         x = {k: torch.from_numpy(v).cuda() for k, v in wl.step_inputs(0).items()}
         y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
-        ts = []
-        for i in range(reps + 3):
-            flush.zero_()
-            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s.record(stream)
-            stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
-            e.record(stream)
-            if i >= 3:
-                ts.append((s, e))
-        torch.cuda.synchronize()
-        stq.stq_pool_check(pool, stream)
-        med = statistics.median(s.elapsed_time(e) for s, e in ts) * 1e-3
-        nbytes, _ = workload_info(wl)
-        packed, _ = stq.stq_pool_bytes(pool)
-        out.append({"requests": R, "heads": wl.H, "pool_gb": packed / 1e9, "touched_gb": nbytes / 1e9,
-                    "kernel_us": med * 1e6, "head_steps_per_s": wl.R * wl.H / med,
-                    "gbs": nbytes / med / 1e9, "frac": nbytes / med / 1e9 / peak})
-        pool.close()
+        row = {"requests": R, "heads": wl.H}
+        for tag, bits, sb in (("quant", wl.unit_bits, 4), ("fp32", np.full(wl.H, 32, np.uint8), 0),
+                              ("fp16", np.full(wl.H, 16, np.uint8), 0)):
+            if tag == "quant":
+                pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, bits, wl.row_factor, wl.col_factor)
+            else:
+                pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, bits)
+            ts = []
+            for i in range(reps + 3):
+                flush.zero_()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record(stream)
+                stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
+                e.record(stream)
+                if i >= 3:
+                    ts.append((s, e))
+            torch.cuda.synchronize()
+            stq.stq_pool_check(pool, stream)
+            med = statistics.median(s.elapsed_time(e) for s, e in ts) * 1e-3
+            nbytes, _ = workload_info(wl, bits, sb)
+            packed, _ = stq.stq_pool_bytes(pool)
+            pool.close()
+            torch.cuda.empty_cache()
+            if tag == "quant":
+                row.update({"pool_gb": packed / 1e9, "touched_gb": nbytes / 1e9, "kernel_us": med * 1e6,
+                            "head_steps_per_s": wl.R * wl.H / med, "gbs": nbytes / med / 1e9,
+                            "frac": nbytes / med / 1e9 / peak})
+            else:
+                row.update({f"{tag}_pool_gb": packed / 1e9, f"{tag}_kernel_us": med * 1e6,
+                            f"{tag}_frac": nbytes / med / 1e9 / peak})
+        row["fp32_over_quant"] = row["fp32_kernel_us"] / row["kernel_us"]
+        out.append(row)
         del x, y
         torch.cuda.empty_cache()
     return out
@@ -497,7 +550,13 @@ def layer_loop(stq, flush, layers: int = 48, R: int = 64, reps: int = 20):
     replay.  fused: one decode launch per layer.  split: per layer the readout
     on the main stream and the write-back on a side stream, joined at the end.
     readout_only: the main-stream half alone (pages unchanged), the path that
-    gates the next layer when the write-backs overlap other work."""
+    gates the next layer when the write-backs overlap other work.
+    The *_gemm variants add, after each layer's decode (fused) or readout
+    (split) on the main stream, a stand-in for the rest of the layer: a bf16
+    projection [R, 5120] x [5120, 5120] with its own weights per layer (read
+    from HBM, as decode-time projections are); gemm_only is that work alone.
+    split_gemm below fused_gemm means the side-stream write-backs are hidden
+    behind it."""
     import torch
     wls = [synth.make_workload(4, R=R, H=16, seed=l) for l in range(layers)]
     pools, idx, xs, ys, us = [], [], [], [], []
@@ -511,21 +570,28 @@ def layer_loop(stq, flush, layers: int = 48, R: int = 64, reps: int = 20):
         ys.append(torch.empty((w.R, w.H, 128), dtype=torch.float32, device="cuda"))
         us.append(torch.empty((w.R, w.H, 128), dtype=torch.float32, device="cuda"))
     main, side = torch.cuda.Stream(), torch.cuda.Stream()
+    hidden = 5120
+    act = torch.randn((R, hidden), dtype=torch.bfloat16, device="cuda")
+    weights = [torch.randn((hidden, hidden), dtype=torch.bfloat16, device="cuda") * 0.01 for _ in range(layers)]
+    proj = torch.empty((R, hidden), dtype=torch.bfloat16, device="cuda")
 
     def body(kind):
         for l in range(layers):
-            if kind == "fused":
+            if kind.startswith("fused"):
                 stq.stq_decode_step(pools[l], *idx[l], *xs[l], ys[l], main)
-            elif kind == "split":
+            elif kind.startswith("split"):
                 stq.stq_decode_step_split(pools[l], *idx[l], *xs[l], ys[l], us[l], main, side)
-            else:
+            elif kind == "readout_only":
                 stq.stq_decode_readout(pools[l], *idx[l], *xs[l], ys[l], us[l], main)
-        if kind == "split":
+            if "gemm" in kind:
+                torch.mm(act, weights[l], out=proj)
+        if kind.startswith("split"):
             for p in pools:
                 stq.stq_pool_join(p, main)
 
-    out = {"layers": layers, "heads_per_layer": 16, "requests": R, "slots": 5}
-    for kind in ("fused", "split", "readout_only"):
+    out = {"layers": layers, "heads_per_layer": 16, "requests": R, "slots": 5,
+           "gemm": f"bf16 [{R}, {hidden}] x [{hidden}, {hidden}] per layer"}
+    for kind in ("fused", "split", "readout_only", "gemm_only", "fused_gemm", "split_gemm"):
         torch.cuda.synchronize()
         with torch.cuda.stream(main):
             body(kind)  # eager warm-up (sets the kernels' shared-memory attributes)
@@ -551,9 +617,11 @@ def layer_loop(stq, flush, layers: int = 48, R: int = 64, reps: int = 20):
         out[f"{kind}_graph_us"] = med * 1e6
         out[f"{kind}_head_steps_per_s"] = layers * R * 16 / med
         del g
+    out["split_gemm_over_fused_gemm"] = out["split_gemm_graph_us"] / out["fused_gemm_graph_us"]
     for p in pools:
         stq.stq_pool_check(p)
         p.close()
+    del weights
     torch.cuda.empty_cache()
     return out
 
@@ -562,10 +630,13 @@ def drift(stq, steps: int = 8192, every: int = 512, tokens: int = 256):
     """Long-generation drift: 32 requests x 32 heads, alpha ~ U(0.95, 0.9999),
     GDN at INT4 / INT6 / INT8 and KDA at 6-bit mixed widths (decay per row in
     the same range), each advanced `steps` tokens next to the unquantized fp32
-    recurrence (a raw fp32 pool) on the same inputs; every `every` steps the
+    recurrence (a raw fp32 pool) on the same inputs.  Every `every` steps the
     relative state error ||S^ - S||_F / ||S||_F and readout error
-    ||y^ - y|| / ||y|| per (request, head) are recorded (mean and max).  The
-    inputs of `tokens` distinct steps are cycled."""
+    ||y^ - y|| / ||y|| per (request, head) are taken; the record keeps, per
+    case, the mean and max of the last checkpoint, the largest mean and max
+    over all checkpoints, and (KDA) the last checkpoint's mean state error
+    over the rows of each width.  The inputs of `tokens` distinct steps are
+    cycled (a periodic input after the first `tokens` steps)."""
     import dataclasses
     import torch
     cases = [(f"gdn_int{b}", synth.make_workload(5, bits=b)) for b in (4, 6, 8)]
@@ -587,7 +658,9 @@ def drift(stq, steps: int = 8192, every: int = 512, tokens: int = 256):
         yf = torch.empty_like(yq)
         Sq = torch.empty((wl.R, wl.H, 128, 128), dtype=torch.float32, device="cuda")
         Sf = torch.empty_like(Sq)
-        rec = {"state_rel_err_mean": [], "state_rel_err_max": [], "y_rel_err_mean": [], "y_rel_err_max": []}
+        width = torch.from_numpy(wl.row_bits().astype(np.int64)).cuda()  # [H, 128]
+        es_mean, es_max, ey_mean, ey_max = [], [], [], []
+        by_width = {}
         for t in range(steps):
             x = xs[t % tokens]
             stq.stq_decode_step(pq, req, slot, *x, yq)
@@ -598,12 +671,26 @@ def drift(stq, steps: int = 8192, every: int = 512, tokens: int = 256):
                 es = (torch.linalg.vector_norm(Sq - Sf, dim=(2, 3)) /
                       torch.linalg.vector_norm(Sf, dim=(2, 3)).clamp_min(1e-30))
                 ey = torch.linalg.vector_norm(yq - yf, dim=2) / torch.linalg.vector_norm(yf, dim=2).clamp_min(1e-30)
-                rec["state_rel_err_mean"].append(float(es.mean()))
-                rec["state_rel_err_max"].append(float(es.max()))
-                rec["y_rel_err_mean"].append(float(ey.mean()))
-                rec["y_rel_err_max"].append(float(ey.max()))
+                es_mean.append(float(es.mean()))
+                es_max.append(float(es.max()))
+                ey_mean.append(float(ey.mean()))
+                ey_max.append(float(ey.max()))
+                if wl.kind == synth.KDA and t + 1 == steps:
+                    d2 = ((Sq - Sf) ** 2).sum(dim=3)  # [R, H, 128] per row
+                    f2 = (Sf ** 2).sum(dim=3)
+                    for b in (4, 6, 8):
+                        m = (width == b).unsqueeze(0)
+                        num = (d2 * m).sum(dim=2).sqrt()
+                        den = (f2 * m).sum(dim=2).sqrt().clamp_min(1e-30)
+                        by_width[str(b)] = float((num / den).mean())
         stq.stq_pool_check(pq)
         stq.stq_pool_check(pf)
+        rec = {"state_rel_err_mean": es_mean[-1], "state_rel_err_max": es_max[-1],
+               "y_rel_err_mean": ey_mean[-1], "y_rel_err_max": ey_max[-1],
+               "state_rel_err_mean_peak": max(es_mean), "state_rel_err_max_peak": max(es_max),
+               "y_rel_err_max_peak": max(ey_max), "checkpoints": len(es_mean)}
+        if by_width:
+            rec["state_rel_err_mean_by_row_width"] = by_width
         out["cases"][name] = rec
         pq.close()
         pf.close()

@@ -37,7 +37,13 @@
  *   - Setting the environment variable STQ_FAULT=alloc makes
  *     stq_pool_create fail with STQ_ERR_OOM, STQ_FAULT=launch makes every
  *     launching call fail with STQ_ERR_CUDA, both before any CUDA call
- *     (host-side fault injection for tests).
+ *     (host-side fault injection for tests).  STQ_FAULT=timeout exercises the
+ *     decode kernel's bounded waits: calls made while it is set shorten the
+ *     wait limit from 1 s to 2 ms and make the first stage of the first CTA
+ *     expect 16 bytes more than its copies deliver, so that every copy lands
+ *     and that wait runs out; the kernel then waits (bounded) for its copies,
+ *     returns, and stq_pool_check reports STQ_ERR_TIMEOUT.  The step's
+ *     results are then undefined for the tiles that CTA did not finish.
  */
 #ifndef STQ_H
 #define STQ_H
@@ -244,8 +250,10 @@ stq_status stq_decode_step_split(stq_pool *pool, const int32_t *req_idx,
  * process exits).  It never allocates or frees memory.
  *   - n * H may be at most 8192 tiles (n * H * 128 floats <= 2^20);
  *     larger calls return STQ_ERR_ARG before anything is enqueued.
- *   - The first call on a device looks up the array's device address (once
- *     per device); make that first call before any stream capture.
+ *   - The first call on a device looks up the array's device address on
+ *     that device; make that first call before any stream capture.  Later
+ *     calls look it up again (so a context re-created after a device reset
+ *     is served from its own copy).
  *   - All calls on a device share the one array: calls that may overlap on the
  *     GPU (other streams, other threads) race on it and must be serialized by
  *     the caller.  Each call writes the array in full before reading it, so
@@ -283,6 +291,31 @@ stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const 
 stq_status stq_decode_step_host(stq_pool *pool, const int32_t *req_idx, const int32_t *slot_idx,
                                 int32_t n, const float *q, const float *k, const float *v,
                                 const float *beta, const float *gate, float *y, void *stream);
+
+/*
+ * The host-buffer step with every input in ONE host block, so that the inputs
+ * cross the bus in a single copy (no counterpart in the paper).
+ *
+ * stq_host_block_layout: for n entries of `pool`, the byte offsets inside
+ * the block of req_idx, slot_idx, q, k, v, beta and gate, in that order, in
+ * offsets[0..6] (each a multiple of 256, arrays as stq_decode_step lays them
+ * out: int32 [n], int32 [n], fp32 [n][H][128] x 3, fp32 [n][H], gate fp32
+ * [n][H] (GDN) or [n][H][128] (KDA)), and the block size in *bytes (the end
+ * of the gate array).  The bytes between arrays are never read.  STQ_ERR_ARG
+ * for a NULL pool or output, or n < 0.
+ *
+ * stq_decode_step_host_block: stq_decode_step_host with the inputs read
+ * from `block` (host memory of at least `bytes` bytes, as laid out above for
+ * this n; `bytes` must equal the layout's size, else STQ_ERR_ARG) and y
+ * written to the host array y (fp32 [n][H][128]).  One host-to-device copy
+ * of the block, the step, one device-to-host copy of y, all on `stream`;
+ * the results equal stq_decode_step's bit for bit, and the staging rules
+ * (shared buffer, first-call allocation, page-locked memory for
+ * asynchronous copies) are those of stq_decode_step_host.
+ */
+stq_status stq_host_block_layout(const stq_pool *pool, int32_t n, size_t offsets[7], size_t *bytes);
+stq_status stq_decode_step_host_block(stq_pool *pool, int32_t n, const void *block, size_t bytes, float *y,
+                                      void *stream);
 
 /* Make `stream` wait for the pool's pending split write-back (no-op if none). */
 stq_status stq_pool_join(stq_pool *pool, void *stream);

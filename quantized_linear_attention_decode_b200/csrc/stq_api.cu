@@ -132,10 +132,6 @@ stq_status check_desc(const stq_pool_desc *d, std::vector<uint8_t> *row_bits)
             if (d->unit_bits[u] == 32)
                 return fail(STQ_ERR_UNSUPPORTED, "unit_bits[%zu] = 32: fp32 units must make up the whole pool", u);
     if (raw && d->flags != 0) return fail(STQ_ERR_ARG, "a raw pool has no scales (flags must be 0)");
-    if (d->flags & STQ_FIT_COLUMNS)
-        for (size_t u = 0; u < nunits; ++u)
-            if (d->unit_bits[u] == 16)
-                return fail(STQ_ERR_UNSUPPORTED, "STQ_FIT_COLUMNS with FP16 pivot units (unit_bits[%zu] = 16)", u);
     if ((d->flags & STQ_FIT_COLUMNS) && d->row_weight)
         for (size_t e = 0; e < (size_t)H * stq::kD; ++e)
             if (!(std::isfinite(d->row_weight[e]) && d->row_weight[e] > 0.0f))
@@ -196,6 +192,10 @@ stq::PoolView view(stq_pool *p)
     v.fit = p->fit ? 1 : 0;
     v.t = p->t;
     v.err = p->d_err;
+    // STQ_FAULT=timeout: a wait that nothing completes, given a short limit
+    const bool stall = fault("timeout");
+    v.wait_ns = stall ? 2000000ull : 1000000000ull;
+    v.stall_tx = stall ? 16u : 0u;
     return v;
 }
 
@@ -675,15 +675,23 @@ constexpr int kMaxScratchDevices = 64;
 float *g_static_u_tilde_ptr[kMaxScratchDevices] = {};
 std::mutex g_static_mu;
 
-// Device address of the array on the current device, looked up once per
-// device.  In host code the array's name only stands for the symbol.
-cudaError_t static_u_tilde(int dev, float **out)
+// Device address of the array on the current device.  In host code the
+// array's name only stands for the symbol.  Outside stream capture the
+// address is looked up on every call (so a context re-created after a device
+// reset gets its own image's address) and cached per device; a call made
+// while `stream` is being captured uses the cached address, which an earlier
+// uncaptured call on this device must have set.
+cudaError_t static_u_tilde(int dev, cudaStream_t stream, float **out)
 {
     if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+    if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (g_static_u_tilde_ptr[dev] == nullptr) {
+    if (cs == cudaStreamCaptureStatusNone || g_static_u_tilde_ptr[dev] == nullptr) {
+        if (cs != cudaStreamCaptureStatusNone) return cudaErrorStreamCaptureUnsupported;
         void *ptr = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_u_tilde);
+        e = cudaGetSymbolAddress(&ptr, g_static_u_tilde);
         if (e != cudaSuccess) return e;
         g_static_u_tilde_ptr[dev] = static_cast<float *>(ptr);
     }
@@ -711,10 +719,10 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
     DeviceGuard g(p->device);
     NvtxRange nvtx("stq_decode_step_static");
     if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
-    float *u = nullptr;
-    cudaError_t e = static_u_tilde(p->device, &u);
-    if (e != cudaSuccess) return cuda_fail(e, "address of the built-in scratch");
     const cudaStream_t s0 = (cudaStream_t)stream;
+    float *u = nullptr;
+    cudaError_t e = static_u_tilde(p->device, s0, &u);
+    if (e != cudaSuccess) return cuda_fail(e, "address of the built-in scratch");
     e = join_async(p, s0);
     if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
     e = debug_checks(p, req_idx, slot_idx, n, s0);
@@ -742,9 +750,10 @@ namespace {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Byte offsets of the staged arrays for n entries (each 256-byte aligned).
+// Byte offsets of the staged arrays for n entries (each 256-byte aligned);
+// the inputs end at `inputs`, y follows.
 struct HostLayout {
-    size_t req, slot, q, k, v, beta, gate, y, total;
+    size_t req, slot, q, k, v, beta, gate, inputs, y, total;
 };
 
 HostLayout host_layout(const stq_pool *p, int32_t n)
@@ -758,7 +767,9 @@ HostLayout host_layout(const stq_pool *p, int32_t n)
     L.k = o;    o += align256(vec);
     L.v = o;    o += align256(vec);
     L.beta = o; o += align256(per);
-    L.gate = o; o += align256(p->kind == STQ_KDA ? vec : per);
+    L.gate = o; o += p->kind == STQ_KDA ? vec : per;
+    L.inputs = o;
+    o = align256(o);
     L.y = o;    o += align256(vec);
     L.total = o;
     return L;
@@ -786,6 +797,26 @@ cudaError_t host_staging(stq_pool *p, size_t bytes, cudaStream_t stream)
     // the previous call may have run on another stream: wait for it unless it is done
     if (p->h_used && cudaEventQuery(p->h_done) != cudaSuccess) e = cudaStreamWaitEvent(stream, p->h_done, 0);
     return e;
+}
+
+// The step on inputs already copied into the staging buffer (queued on s0),
+// then y copied back to the host; records the pool's staging event.
+stq_status host_decode_and_copy_out(stq_pool *p, int32_t n, const HostLayout &L, float *y, cudaStream_t s0)
+{
+    uint8_t *d = p->h_stage;
+    const size_t vec = (size_t)n * p->H * kD * sizeof(float);
+    const stq::DecodeIO io{reinterpret_cast<const int32_t *>(d + L.req), reinterpret_cast<const int32_t *>(d + L.slot),
+                           n, reinterpret_cast<const float *>(d + L.q), reinterpret_cast<const float *>(d + L.k),
+                           reinterpret_cast<const float *>(d + L.v), reinterpret_cast<const float *>(d + L.beta),
+                           reinterpret_cast<const float *>(d + L.gate), reinterpret_cast<float *>(d + L.y), nullptr};
+    cudaError_t e = debug_checks(p, io.req_idx, io.slot_idx, n, s0);
+    if (e == cudaSuccess) e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
+    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
+    const cudaError_t eo = e == cudaSuccess ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
+    const cudaError_t er = cudaEventRecord(p->h_done, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (eo != cudaSuccess) return cuda_fail(eo, "host-decode output copy");
+    return er == cudaSuccess ? STQ_OK : cuda_fail(er, "host-decode event");
 }
 
 }  // namespace
@@ -828,18 +859,49 @@ stq_status stq_decode_step_host(stq_pool *p, const int32_t *req_idx, const int32
         cudaEventRecord(p->h_done, s0);
         return cuda_fail(e, "host-decode input copy");
     }
-    const stq::DecodeIO io{reinterpret_cast<const int32_t *>(d + L.req), reinterpret_cast<const int32_t *>(d + L.slot),
-                           n, reinterpret_cast<const float *>(d + L.q), reinterpret_cast<const float *>(d + L.k),
-                           reinterpret_cast<const float *>(d + L.v), reinterpret_cast<const float *>(d + L.beta),
-                           reinterpret_cast<const float *>(d + L.gate), reinterpret_cast<float *>(d + L.y), nullptr};
-    e = debug_checks(p, io.req_idx, io.slot_idx, n, s0);
-    if (e == cudaSuccess) e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
-    if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
-    const cudaError_t eo = e == cudaSuccess ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
-    const cudaError_t er = cudaEventRecord(p->h_done, s0);
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-    if (eo != cudaSuccess) return cuda_fail(eo, "host-decode output copy");
-    return er == cudaSuccess ? STQ_OK : cuda_fail(er, "host-decode event");
+    return host_decode_and_copy_out(p, n, L, y, s0);
+}
+
+stq_status stq_host_block_layout(const stq_pool *p, int32_t n, size_t offsets[7], size_t *bytes)
+{
+    if (p == nullptr || offsets == nullptr || bytes == nullptr) return fail(STQ_ERR_ARG, "NULL argument");
+    if (n < 0) return fail(STQ_ERR_ARG, "n = %d", n);
+    if ((long long)n * p->H > 0x7FFFFFFFll) return fail(STQ_ERR_ARG, "n * H too large");
+    const HostLayout L = host_layout(p, n);
+    const size_t o[7] = {L.req, L.slot, L.q, L.k, L.v, L.beta, L.gate};
+    for (int a = 0; a < 7; ++a) offsets[a] = o[a];
+    *bytes = L.inputs;
+    return STQ_OK;
+}
+
+stq_status stq_decode_step_host_block(stq_pool *p, int32_t n, const void *block, size_t bytes, float *y,
+                                      void *stream)
+{
+    if (p == nullptr) return fail(STQ_ERR_ARG, "pool is NULL");
+    if (n < 0) return fail(STQ_ERR_ARG, "n = %d", n);
+    if ((long long)n * p->H > 0x7FFFFFFFll) return fail(STQ_ERR_ARG, "n * H too large");
+    if (n > 0 && (block == nullptr || y == nullptr)) return fail(STQ_ERR_ARG, "block or y is NULL");
+    const HostLayout L = host_layout(p, n);
+    if (bytes != L.inputs)
+        return fail(STQ_ERR_ARG, "block of %zu bytes; the layout for n = %d takes %zu", bytes, n, L.inputs);
+    if (n == 0) return STQ_OK;
+    if (fault("launch")) return fail(STQ_ERR_CUDA, "injected launch failure (STQ_FAULT=launch)");
+    DeviceGuard g(p->device);
+    NvtxRange nvtx("stq_decode_step_host_block");
+    if (!g.ok) return fail(STQ_ERR_CUDA, "cannot select device %d", p->device);
+    const cudaStream_t s0 = (cudaStream_t)stream;
+    cudaError_t e = host_staging(p, L.total, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "host-decode staging");
+    e = join_async(p, s0);
+    if (e != cudaSuccess) return cuda_fail(e, "wait for the pending write-back");
+    uint8_t *d = p->h_stage;
+    p->h_used = true;
+    e = cudaMemcpyAsync(d, block, L.inputs, cudaMemcpyHostToDevice, s0);
+    if (e != cudaSuccess) {
+        cudaEventRecord(p->h_done, s0);
+        return cuda_fail(e, "host-decode input copy");
+    }
+    return host_decode_and_copy_out(p, n, L, y, s0);
 }
 
 stq_status stq_pool_join(stq_pool *p, void *stream)

@@ -50,7 +50,6 @@ constexpr int kWriteback = 2;  // steps 4-7 given u~: requantise and pack in pla
 constexpr int kStages = 4;
 constexpr int kRedStride = 288;  // floats per warp in red: 256 column partials, or the padded row-max exchange
 constexpr int kMaxPage = kMaxStagedPage;               // 16896: every row at 8 bits
-constexpr unsigned long long kWaitNs = 1000000000ull;  // bounded waits give up after 1 s
 
 struct __align__(128) Stage {
     uint8_t page[kMaxPage];
@@ -158,12 +157,14 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t 
     return ok != 0;
 }
 
-__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long *bar, uint32_t parity)
+// Waits for the phase of parity `parity`; gives up (false) after limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(unsigned long long *bar, uint32_t parity,
+                                                  unsigned long long limit_ns)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > kWaitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     return true;
 }
 
@@ -440,12 +441,26 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
     float2 av[4], ay[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) av[p] = ay[p] = make_float2(0.0f, 0.0f);
+    // a fitted page's pivot rows hold X / r: their values enter as mu / c_j, like codes
+    float2 ic[4];
+    if (B == 0 && FIT) {
+        const float4 a = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg);
+        const float4 b = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg + 16);
+        ic[0] = make_float2(rcp_approx(a.x), rcp_approx(a.y));
+        ic[1] = make_float2(rcp_approx(a.z), rcp_approx(a.w));
+        ic[2] = make_float2(rcp_approx(b.x), rcp_approx(b.y));
+        ic[3] = make_float2(rcp_approx(b.z), rcp_approx(b.w));
+    }
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
         if (B != 0 && PR) Codec<B == 0 ? 8 : B>::unpack(S.page + R.off[i], cg, z[ii]);
         else if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
         else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
+        if (B == 0 && FIT && R.bits[i] == 16) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) z[ii][p] = fmul2(z[ii][p], ic[p]);
+        }
         if constexpr (ACC) {
             const float4 kl = R.kl[i];
 #pragma unroll
@@ -589,7 +604,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
 // groups of the half-warp through shared memory), new scale, requantise,
 // store codes and scales to the page in global memory.
 template <int B, int SB, bool FIT, bool PR = false>
-__device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4])
+__device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S, float2 z[8][4])
 {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -729,11 +744,21 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, float2 z[8][4]
         const int i = i0 + ii;
         const int b = B != 0 ? B : R.bits[i];
         if (B == 0 && b == 16) {
-            // pivot row: mu = X / (r c) = (e / r) w, with R.mrq = e / r for a pivot row
+            // pivot row: mu = X / (r c) = (e / r) w, with R.mrq = e / r for a pivot row; a
+            // fitted page's pivot row keeps mu = X / r = c_j (e / r) w (c_j: the factors
+            // this tile's codes were taken with, still in the stage)
             const float2 m2 = make_float2(R.mrq[i], R.mrq[i]);
             float2 t[4];
 #pragma unroll
             for (int p = 0; p < 4; ++p) t[p] = fmul2(z[ii][p], m2);
+            if (FIT) {
+                const float4 a = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg);
+                const float4 b = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg + 16);
+                t[0] = fmul2(t[0], make_float2(a.x, a.y));
+                t[1] = fmul2(t[1], make_float2(a.z, a.w));
+                t[2] = fmul2(t[2], make_float2(b.x, b.y));
+                t[3] = fmul2(t[3], make_float2(b.z, b.w));
+            }
             Pivot16::store(page + R.off[i], cg, t);
             continue;
         }
@@ -818,7 +843,7 @@ __device__ __forceinline__ TileRef resolve(const PoolView &p, const TileRaw &r)
 }
 
 template <int KIND>
-__device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const TileRef &t)
+__device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const TileRef &t, uint32_t stall_tx = 0)
 {
     Stage &S = sm.st[s];
     sm.stage_page[s] = t.page;
@@ -831,7 +856,8 @@ __device__ __forceinline__ void issue(Smem &sm, int s, const PoolView &p, const 
         mbar_arrive(&sm.full[s]);  // completes the phase with no data; the tile is skipped
         return;
     }
-    mbar_arrive_expect_tx(&sm.full[s], t.bytes + kHeadBlock);
+    // stall_tx (a test hook, 0 otherwise): bytes that no copy delivers, so that the wait runs out
+    mbar_arrive_expect_tx(&sm.full[s], t.bytes + kHeadBlock + stall_tx);
     bulk_load(S.page, t.page, t.bytes, &sm.full[s]);
     bulk_load(S.r, p.t.block + static_cast<size_t>(t.h) * kHeadBlock, kHeadBlock, &sm.full[s]);
 }
@@ -937,13 +963,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
     __syncthreads();  // barriers initialised, locations in
     if (tid == 0)
         for (int a = 0; a < 3; ++a)
-            if (first + a * G < tiles) issue<KIND>(sm, a, p, resolve(p, raw_from_smem(sm, a)));
+            if (first + a * G < tiles)
+                issue<KIND>(sm, a, p, resolve(p, raw_from_smem(sm, a)), first == 0 && a == 0 ? p.stall_tx : 0u);
     cp_async_wait<0>();
     __syncthreads();  // the first vectors and the stages' validity are visible
     bool timed_out = false;
     if (tid >= kD) {
         // warp-uniform outcome: row_setup's shuffles need every lane
-        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0))) row_setup<KIND, SB, MODE, FIT>(sm, sm.st[0], sm.rc[0], 0);
+        if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[0], 0, p.wait_ns))) row_setup<KIND, SB, MODE, FIT>(sm, sm.st[0], sm.rc[0], 0);
         else timed_out = true;
     }
     timed_out = __syncthreads_or(timed_out) != 0;
@@ -996,7 +1023,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
             }
         } else if (tile + G < tiles) {
             const int sn = (i + 1) % kStages;
-            if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1)))
+            if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1, p.wait_ns)))
                 row_setup<KIND, SB, MODE, FIT>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
             else
                 tout = true;
@@ -1005,14 +1032,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         if (valid && MODE != kReadout) {
             if constexpr (KIND == STQ_KDA) {
                 const int wb = R.wbits[tid >> 5];
-                if (wb == 6) pass2<6, SB, FIT, true>(sm, R, z);
-                else if (wb == 8) pass2<8, SB, FIT, true>(sm, R, z);
-                else if (wb == 4) pass2<4, SB, FIT, true>(sm, R, z);
-                else pass2<0, SB, FIT>(sm, R, z);
+                if (wb == 6) pass2<6, SB, FIT, true>(sm, R, S, z);
+                else if (wb == 8) pass2<8, SB, FIT, true>(sm, R, S, z);
+                else if (wb == 4) pass2<4, SB, FIT, true>(sm, R, S, z);
+                else pass2<0, SB, FIT>(sm, R, S, z);
             }
-            else if (b == 8) pass2<8, SB, FIT>(sm, R, z);
-            else if (b == 6) pass2<6, SB, FIT>(sm, R, z);
-            else pass2<4, SB, FIT>(sm, R, z);
+            else if (b == 8) pass2<8, SB, FIT>(sm, R, S, z);
+            else if (b == 6) pass2<6, SB, FIT>(sm, R, S, z);
+            else pass2<4, SB, FIT>(sm, R, S, z);
         }
     }
     if (FIT && MODE != kReadout) {
@@ -1029,7 +1056,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
             atomicOr(p.err, kErrTimeout);
             for (int k = i; k < i + 3; ++k) {
                 const int t = first + k * G;
-                if (t < tiles) mbar_wait_bounded(&sm.full[k % kStages], (k / kStages) & 1);
+                if (t < tiles) mbar_wait_bounded(&sm.full[k % kStages], (k / kStages) & 1, p.wait_ns);
             }
         }
         if (sm.flags) atomicOr(p.err, sm.flags);

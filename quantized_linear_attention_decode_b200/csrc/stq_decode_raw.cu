@@ -10,8 +10,10 @@
 // y = P^T q + (k.q) u, so one pass over S forms both column sums.
 //
 // The same kernel advances the GDN FP16 pivot heads of a quantized pool
-// (PIVOT): their page keeps the pool's scale section (slots of 1) and stores
-// mu = X / (r c) in binary16, so with P = g S and S_ij = r_i c_j mu_ij
+// (PIVOT): their page keeps the pool's scale section (slots of 1; in a fitted
+// pool also its column factor section, unused) and stores mu = X / (r c) in
+// binary16 (mu = X / r in a fitted pool: c_j = 1 below), so with P = g S and
+// S_ij = r_i c_j mu_ij
 //   column sums over (g k r)_i mu_ij and (g q r)_i mu_ij, times c_j;
 //   mu'_ij = g mu_ij + (k_i / r_i) (u_j / c_j).
 // CTAs of the other heads return at once.
@@ -123,7 +125,7 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
         return;
     }
     uint8_t *page = p.pages + (static_cast<size_t>(req) * p.S + slot) * p.slot_bytes + p.t.head_off[h] +
-                    (PIVOT ? p.scale_bytes * kD : 0);
+                    (PIVOT ? p.scale_bytes * kD + (p.fit ? kFitBytes : 0) : 0);
     const size_t vec = static_cast<size_t>(tile) * kD;
     const int warp = tid >> 5, lane = tid & 31;
     const int rgl = lane >> 4, cg = lane & 15;
@@ -190,7 +192,7 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
             yz += red[w][1][j];
         }
         const float kq = (kqp[0] + kqp[1]) + (kqp[2] + kqp[3]);
-        const float cj = PIVOT ? p.t.c[h * kD + j] : 1.0f;
+        const float cj = PIVOT && !p.fit ? p.t.c[h * kD + j] : 1.0f;  // a fitted page's pivots leave c out
         const float u = io.beta[tile] * (io.v[vec + j] - (PIVOT ? cj * vz : vz));
         const float yj = fmaf(kq, u, PIVOT ? cj * yz : yz);
         io.y[vec + j] = yj;

@@ -56,6 +56,8 @@ struct PoolView {
     int fit;             // nonzero: pages carry column factors refitted at every quantisation
     Tables t;
     uint32_t *err;
+    unsigned long long wait_ns;  // limit of every bounded device-side wait
+    uint32_t stall_tx;           // test hook: bytes the first stage of CTA 0 expects beyond its copies
 };
 
 struct DecodeIO {

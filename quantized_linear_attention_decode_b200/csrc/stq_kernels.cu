@@ -35,11 +35,12 @@ __device__ __forceinline__ uint8_t *tile_page(const PoolView &p, int req, int sl
 
 // fp32 state -> packed page: mu = fl32(S / (r c)) (fp64 quotient), s = fl32(max|mu| / q_b),
 // z = clip(rint(fl32(mu / s)), -q_b, q_b).  A 16-bit row is an FP16 pivot: its scale
-// slot holds 1 and it stores mu rounded once to binary16.  With fitted column
-// factors the codes are taken with the table's c, then every column is refitted
-// in fp64, c_j = sum_i w_i^2 v_ij S_ij / sum_i w_i^2 v_ij^2 with v_ij = s_i r_i z_ij
-// (each term formed in the oracle's operation order), and stored in the page.
-// One warp per row.
+// slot holds 1 and it stores mu rounded once to binary16 (in a fitted page
+// mu = fl32(S / r), without the column factor).  With fitted column factors the
+// codes are taken with the table's c, then every column is refitted over the
+// non-pivot rows in fp64, c_j = sum_i w_i^2 v_ij S_ij / sum_i w_i^2 v_ij^2 with
+// v_ij = s_i r_i z_ij (each term formed in the oracle's operation order), and
+// stored in the page.  One warp per row.
 __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t *req_idx,
                                                        const int32_t *slot_idx, const float *state)
 {
@@ -67,9 +68,10 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
         const float x[4] = {x4.x, x4.y, x4.z, x4.w};
         float mu[4];
         float a = 0.0f;
+        const bool pivot_fit = b == 16 && p.fit;  // a fitted page's pivot row leaves c out
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            mu[t] = static_cast<float>(static_cast<double>(x[t]) / (r * static_cast<double>(cj[t])));
+            mu[t] = static_cast<float>(static_cast<double>(x[t]) / (pivot_fit ? r : r * static_cast<double>(cj[t])));
             a = fmaxf(a, fabsf(mu[t]));
             bad |= !isfinite(x[t]);
         }
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(PoolView p, const int32_t
 }
 
 // packed page -> fp32 reconstruction fl32(((s r) c) z) computed in fp64 (z: the binary16
-// value of a pivot row).  One warp per row.
+// value of a pivot row, without c in a fitted page).  One warp per row.
 __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32_t *req_idx,
                                                          const int32_t *slot_idx, float *state)
 {
@@ -203,11 +205,12 @@ __global__ void __launch_bounds__(256) dequantize_kernel(PoolView p, const int32
 #pragma unroll
             for (int t = 0; t < 4; ++t) zz[t] = static_cast<int>(w << (26 - 6 * t)) >> 26;
         }
+        const bool pivot_fit = b == 16 && p.fit;  // a fitted page's pivot row leaves c out
         float4 o;
-        o.x = static_cast<float>(sr * static_cast<double>(cj[0]) * zz[0]);
-        o.y = static_cast<float>(sr * static_cast<double>(cj[1]) * zz[1]);
-        o.z = static_cast<float>(sr * static_cast<double>(cj[2]) * zz[2]);
-        o.w = static_cast<float>(sr * static_cast<double>(cj[3]) * zz[3]);
+        o.x = static_cast<float>(sr * (pivot_fit ? 1.0 : static_cast<double>(cj[0])) * zz[0]);
+        o.y = static_cast<float>(sr * (pivot_fit ? 1.0 : static_cast<double>(cj[1])) * zz[1]);
+        o.z = static_cast<float>(sr * (pivot_fit ? 1.0 : static_cast<double>(cj[2])) * zz[2]);
+        o.w = static_cast<float>(sr * (pivot_fit ? 1.0 : static_cast<double>(cj[3])) * zz[3]);
         *reinterpret_cast<float4 *>(S + i * kD + lane * 4) = o;
     }
 }

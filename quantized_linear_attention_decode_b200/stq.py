@@ -27,7 +27,8 @@ STQ_OK, STQ_ERR_ARG, STQ_ERR_OOM, STQ_ERR_CUDA, STQ_ERR_INDEX, STQ_ERR_NONFINITE
 EXPORTS = ("stq_pool_create", "stq_pool_destroy", "stq_pool_bytes", "stq_desc_bytes",
            "stq_page_layout", "stq_quantize_state", "stq_dequantize_state", "stq_decode_step",
            "stq_decode_readout", "stq_decode_writeback", "stq_decode_step_split", "stq_pool_join",
-           "stq_decode_step_static", "stq_decode_step_host", "stq_lifetime_weight", "stq_allocate_bits",
+           "stq_decode_step_static", "stq_decode_step_host", "stq_host_block_layout",
+           "stq_decode_step_host_block", "stq_lifetime_weight", "stq_allocate_bits",
            "stq_export_slot", "stq_import_slot", "stq_pool_check", "stq_launch_count",
            "stq_status_str", "stq_last_error")
 
@@ -68,6 +69,8 @@ def load():
         "stq_dequantize_state": [P, P, P, I32, P, P],
         "stq_decode_step": [P, P, P, I32, P, P, P, P, P, P, P],
         "stq_decode_step_host": [P, P, P, I32, P, P, P, P, P, P, P],
+        "stq_host_block_layout": [P, I32, P, P],
+        "stq_decode_step_host_block": [P, I32, P, SZ, P, P],
         "stq_decode_readout": [P, P, P, I32, P, P, P, P, P, P, P, P],
         "stq_decode_writeback": [P, P, P, I32, P, P, P, P],
         "stq_decode_step_split": [P, P, P, I32, P, P, P, P, P, P, P, P, P],
@@ -262,6 +265,27 @@ def stq_decode_step_host(pool: Pool, req_idx, slot_idx, q, k, v, beta, gate, y, 
         n, _host(q, f, vec, "q"), _host(k, f, vec, "k"), _host(v, f, vec, "v"),
         _host(beta, f, (n, pool.H), "beta"), _host(gate, f, gshape, "gate"), _host(y, f, vec, "y"),
         _stream(stream)))
+
+
+def stq_host_block_layout(pool: Pool, n: int):
+    """(offsets of req_idx, slot_idx, q, k, v, beta, gate; block bytes) of the
+    one-block host layout for n entries."""
+    offs = (C.c_size_t * 7)()
+    nb = C.c_size_t()
+    _check(load().stq_host_block_layout(pool.handle, int(n), offs, C.byref(nb)))
+    return [int(o) for o in offs], nb.value
+
+
+def stq_decode_step_host_block(pool: Pool, n: int, block, y, stream=None) -> None:
+    """stq_decode_step_host with every input in one host block (a uint8 CPU
+    tensor laid out by stq_host_block_layout): one copy in, one copy of y out."""
+    import torch
+    if not isinstance(block, torch.Tensor) or block.device.type != "cpu" or block.dtype != torch.uint8 \
+            or not block.is_contiguous():
+        raise TypeError("block must be a contiguous uint8 CPU tensor")
+    vec, _ = _vecs(pool, n)
+    _check(load().stq_decode_step_host_block(pool.handle, int(n), C.c_void_p(block.data_ptr()), block.numel(),
+                                             _host(y, torch.float32, vec, "y"), _stream(stream)))
 
 
 def _vecs(pool, n):

@@ -238,12 +238,13 @@ def make_workload(config: int, seed: int = 0, *, R: int | None = None, H: int | 
     raise ValueError(f"unknown workload {config}")
 
 
-def algorithmic_bytes_per_head_step(kind: int, row_bits_sum: int) -> int:
+def algorithmic_bytes_per_head_step(kind: int, row_bits_sum: int, scale_bytes: int = 4) -> int:
     """HBM bytes one (request, head) decode step must move: packed codes read
-    and written, 128 fp32 scales read and written, q, k, v read, y written,
+    and written, 128 row scales of `scale_bytes` bytes read and written (4:
+    fp32, 2: binary16, 0: a raw fp16 / fp32 state), q, k, v read, y written,
     beta and the gate read."""
     codes = 2 * 16 * row_bits_sum
-    scales = 2 * D * 4
+    scales = 2 * D * scale_bytes
     io = 3 * D * 4 + D * 4 + 4
     gate = 4 if kind == GDN else D * 4
     return codes + scales + io + gate

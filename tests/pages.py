@@ -129,6 +129,7 @@ class Compare:
         self.worst_x = 0.0
         self.worst_c = 0.0
         self.tied_columns = 0
+        self.flip_pages = 0
 
     def y(self, y_gpu, y_ref, where=""):
         y_gpu = np.asarray(y_gpu, np.float64)
@@ -148,6 +149,7 @@ class Compare:
         self.codes += int((~piv).sum()) * D
         qref = np.asarray(quot, np.float64).copy()
         zref = zr.copy()
+        flipped = False
         if fmt & 1:
             # binary16 scales: a row whose s = a / q_b lies next to a rounding midpoint of
             # binary16 may round to the other neighbour on the GPU (its a differs by an ulp
@@ -163,12 +165,18 @@ class Compare:
                 qref[i] = mu / float(sg[i])
                 zref[i] = np.clip(np.rint(qref[i]), -qb, qb)
                 self.flips.append((where, int(i), float(sr[i]), float(sg[i])))
+                flipped = True
         diff = zg != zref
         if fmt & FITC:
             # fitted factors: fp32 sums on the GPU, fp64 in the oracle; a column that holds a
             # near-tie code is refitted from a different code and is logged, not compared
             cg_, cr_ = col_factors(page_gpu, row_bits, fmt), col_factors(page_ref, row_bits, fmt)
             tied = diff.any(axis=0)
+            if flipped:
+                # a row's binary16 scale took the other neighbour: every column was refitted
+                # with that scale, so this page's factors are logged, not compared
+                tied[:] = True
+                self.flip_pages += 1
             rel = np.abs(cg_.astype(np.float64) - cr_) / np.maximum(np.abs(cr_), 1e-30)
             self.worst_c = max(self.worst_c, float(rel[~tied].max()) if (~tied).any() else 0.0)
             self.tied_columns += int(tied.sum())
@@ -243,7 +251,8 @@ class Compare:
               f"scale flips {len(self.flips)}, raw values {self.values}, raw ties {self.raw_ties}, "
               f"worst y rel {self.worst_y:.2e}, worst scale rel {self.worst_s:.2e}, "
               f"worst raw rel {self.worst_x:.2e}, worst column factor rel {self.worst_c:.2e} "
-              f"({self.tied_columns} columns with a near-tie not compared)")
+              f"({self.tied_columns} columns with a near-tie not compared; factors of {self.flip_pages} pages "
+              f"with a scale flip not compared)")
         assert frac <= self.max_tie_frac, f"tie fraction {frac:.3g} above {self.max_tie_frac}"
         rows = self.codes // 128
         assert len(self.flips) <= max(2, 1e-2 * rows), f"{len(self.flips)} scale flips in {rows} rows"

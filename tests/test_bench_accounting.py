@@ -26,6 +26,11 @@ def test_bytes_per_head_step():
     assert f(synth.GDN, 128 * 8) == 16384 * 2 + 1024 + 2048 + 4 + 4 == 35848
     # KDA head of 32 rows at 4, 64 at 6, 32 at 8 bits: 768 bits per column, as a 6-bit head
     assert f(synth.KDA, 32 * 4 + 64 * 6 + 32 * 8) == 12288 * 2 + 1024 + 2048 + 4 + 512 == 28164
+    # binary16 scales: 2 x 256 bytes; raw states (no scales): a binary16 state is 128 x 128 x 16 bits,
+    # an fp32 state 128 x 128 x 32 bits, read and written
+    assert f(synth.GDN, 128 * 6, scale_bytes=2) == 12288 * 2 + 512 + 2048 + 4 + 4 == 27144
+    assert f(synth.GDN, 128 * 16, scale_bytes=0) == 32768 * 2 + 2048 + 4 + 4 == 67592
+    assert f(synth.GDN, 128 * 32, scale_bytes=0) == 65536 * 2 + 2048 + 4 + 4 == 133128
 
 
 def test_bytes_per_launch_of_the_bench_workload():

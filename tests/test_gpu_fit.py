@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle as orc
-from pages import FITC, Compare, col_factors, split_slot
+from pages import FITC, PIVOT, Compare, col_factors, split_slot
 from quantized_linear_attention_decode_b200 import stq, synth
 
 torch = pytest.importorskip("torch")
@@ -39,13 +39,34 @@ def _pool(wl, w, f16=False):
     return pool, req, slot
 
 
-@pytest.mark.parametrize("config, f16", [(2, False), (3, False), (2, True)])
+def _kda_allocated_pivots(R, H, seed):
+    """KDA with per-row widths from the lifetime-aware allocator (6-bit budget over
+    {4, 6, 8} per head, Lagrangian) and its 8 riskiest rows per head kept as FP16
+    pivots, outlier start: the page's KDA setting (pivot rows, column fit)."""
+    wl = synth.make_workload(3, R=R, H=H)
+    rng = np.random.default_rng(seed)
+    ub = []
+    for h in range(H):
+        d = np.exp(rng.uniform(-2, 2, 128))[:, None] * 4.0 ** (-np.arange(3)[None, :])
+        lw = stq.stq_lifetime_weight(np.log(rng.uniform(0.8, 0.9995, 128)), 8192)
+        bits, _ = stq.stq_allocate_bits(np.full(128, 128.0), [4, 6, 8], d, lw, 6.0,
+                                        method=stq.STQ_ALLOC_LAGRANGE, num_pivots=8, pivot_bits=16)
+        assert int(np.count_nonzero(bits == 16)) == 8
+        ub.append(bits)
+    return dataclasses.replace(wl, unit_bits=np.concatenate(ub), init="outlier")
+
+
+@pytest.mark.parametrize("config, f16", [(2, False), (3, False), (2, True), ("kda_pivots", False),
+                                         ("kda_pivots", True)])
 def test_fit_quantize_dequantize(config, f16):
     """Scales and codes bit-exact; the fitted factors (fp64 sums in another order)
-    within 1e-7; the dequantized state uses the page's factors."""
-    wl = dataclasses.replace(synth.make_workload(config, R=2, H=8), init="outlier")
-    w = _weights(wl, config)
-    fmt = FITC | (1 if f16 else 0)
+    within 1e-7; the dequantized state uses the page's factors (pivot rows: none)."""
+    if config == "kda_pivots":
+        wl = _kda_allocated_pivots(2, 8, 5)
+    else:
+        wl = dataclasses.replace(synth.make_workload(config, R=2, H=8), init="outlier")
+    w = _weights(wl, 3 if config == "kda_pivots" else config)
+    fmt = FITC | (1 if f16 else 0) | (PIVOT if config == "kda_pivots" else 0)
     pool, req, slot = _pool(wl, w, f16)
     rb = wl.row_bits()
     r, c, W = wl.row_factor.reshape(wl.H, 128), wl.col_factor.reshape(wl.H, 128), w.reshape(wl.H, 128)
@@ -68,7 +89,7 @@ def test_fit_quantize_dequantize(config, f16):
 
 
 def _teacher_forced(wl, w, steps, f16=False, split=False):
-    fmt = FITC | (1 if f16 else 0)
+    fmt = FITC | (1 if f16 else 0) | (PIVOT if np.any(wl.unit_bits == 16) else 0)
     pool, req, slot = _pool(wl, w, f16)
     rb = wl.row_bits()
     r, c, W = wl.row_factor.reshape(wl.H, 128), wl.col_factor.reshape(wl.H, 128), w.reshape(wl.H, 128)
@@ -166,3 +187,17 @@ def test_fit_zero_start_pages_carry_initial_factors():
             assert not page[:256].any() and not page[256 + 512:].any()
     pool.close()
     _teacher_forced(wl, w, steps=4, f16=True)
+
+
+def test_fit_with_pivot_rows_kda_allocated():
+    """The page's KDA configuration: allocator-chosen per-row widths, 8 FP16 pivot
+    rows per head, column factors fitted over the non-pivot rows; 8 steps."""
+    wl = _kda_allocated_pivots(3, 4, 11)
+    cmp = _teacher_forced(wl, _weights(wl, 6), steps=8)
+    assert cmp.values == 8 * 3 * 4 * 8 * 128
+
+
+def test_fit_with_pivot_rows_split_and_f16():
+    """Pivot rows with the fit through the split step, binary16 scales."""
+    wl = _kda_allocated_pivots(2, 4, 12)
+    _teacher_forced(wl, _weights(wl, 7), steps=5, f16=True, split=True)

@@ -155,3 +155,52 @@ def test_host_decode_scale_and_fit_formats(config, flags):
     """Binary16 scales and fitted column factors go through the host-buffer step unchanged."""
     wl = synth.make_workload(config, R=12, H=8)
     _same_slots(*_run_twins(wl, 3, flags=flags))
+
+
+def _block(pool, n, req, slot, x, pinned=True):
+    """The one-block host layout of stq_host_block_layout, filled."""
+    offs, nbytes = stq.stq_host_block_layout(pool, n)
+    blk = torch.zeros(nbytes, dtype=torch.uint8)
+    if pinned:
+        blk = blk.pin_memory()
+    raw = blk.numpy()
+    for o, a in zip(offs, [req, slot] + [x[key] for key in KEYS]):
+        b = np.ascontiguousarray(a).view(np.uint8).reshape(-1)
+        raw[o: o + b.size] = b
+    return blk
+
+
+@pytest.mark.parametrize("config", [2, 3])
+def test_host_block_decode_matches_device_step(config):
+    """The single-copy host block: GDN (per-head gate) and KDA (per-row gate)
+    layouts, a subset of requests, three tokens; y and pages bit for bit."""
+    wl = synth.make_workload(config, R=24)
+    ref, got = _pool(wl), _pool(wl)
+    offs, nbytes = stq.stq_host_block_layout(got, 0)
+    assert nbytes == 0 or all(o % 256 == 0 for o in offs)
+    for t in range(3):
+        sel = np.arange(t, wl.R, 2)
+        n = len(sel)
+        inp = wl.step_inputs(t)
+        req = sel.astype(np.int32)
+        slot = wl.slot_of_request[sel].astype(np.int32)
+        x = {key: np.ascontiguousarray(inp[key][sel]) for key in KEYS}
+        y_ref = torch.empty((n, wl.H, 128), dtype=torch.float32, device="cuda")
+        stq.stq_decode_step(ref, _cuda(req), _cuda(slot), *[_cuda(x[key]) for key in KEYS], y_ref)
+        blk = _block(got, n, req, slot, x)
+        offs, nbytes = stq.stq_host_block_layout(got, n)
+        assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and blk.numel() == nbytes
+        y_got = torch.full((n, wl.H, 128), float("nan")).pin_memory()
+        stq.stq_decode_step_host_block(got, n, blk, y_got)
+        torch.cuda.current_stream().synchronize()
+        stq.stq_pool_check(ref)
+        stq.stq_pool_check(got)
+        np.testing.assert_array_equal(y_got.numpy(), y_ref.cpu().numpy())
+    _same_slots(_slots(ref, wl), _slots(got, wl))
+    # a block of the wrong size is refused before anything is queued
+    with pytest.raises(stq.StqError) as e:
+        stq.stq_decode_step_host_block(got, 1, torch.zeros(16, dtype=torch.uint8),
+                                       torch.empty((1, wl.H, 128)))
+    assert e.value.status == stq.STQ_ERR_ARG
+    ref.close()
+    got.close()

@@ -121,7 +121,6 @@ def test_desc_bytes_pivot_pool():
     ([32, 8, 32, 32], 0, "STQ_ERR_UNSUPPORTED"),   # fp32 units among quantized ones
     ([16, 16, 16, 16], 1, "STQ_ERR_ARG"),          # a raw pool has no scales
     ([6, 6, 6, 6], 4, "STQ_ERR_ARG"),              # unknown flag
-    ([16, 6, 8, 6], 2, "STQ_ERR_UNSUPPORTED"),     # fitted column factors with FP16 pivots
     ([16, 16, 16, 16], 2, "STQ_ERR_ARG"),          # a raw pool has no scales or factors
     ([6, 12, 6, 6], 0, "STQ_ERR_ARG"),
 ])
@@ -129,6 +128,18 @@ def test_desc_format_validation(ub, flags, status):
     with pytest.raises(stq.StqError) as e:
         stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, np.array(ub, np.uint8), flags=flags)
     assert stq.STATUS[e.value.status] == status
+
+
+def test_fitted_pool_with_pivots_layout():
+    """FP16 pivot units in a fitted pool: each page keeps its scales, its 128 fp32
+    column factors, and 256 bytes per pivot row (GDN: a whole pivot head)."""
+    bits = np.array([16, 6, 8, 6], np.uint8)
+    _, slot = stq.stq_desc_bytes(stq.STQ_GDN, 1, 1, 4, bits, flags=stq.STQ_FIT_COLUMNS)
+    page = lambda b: (512 + 512 + 16 * 128 * b + 127) // 128 * 128  # noqa: E731
+    assert slot == sum(page(int(b)) for b in bits)
+    kb = np.tile(np.array([16] * 8 + [4] * 120, np.uint8), 2)
+    _, kslot = stq.stq_desc_bytes(stq.STQ_KDA, 1, 1, 2, kb, flags=stq.STQ_FIT_COLUMNS | stq.STQ_SCALE_F16)
+    assert kslot == 2 * ((256 + 512 + 8 * 256 + 120 * 64 + 127) // 128 * 128)
 
 
 def test_unsupported_head_dim():
