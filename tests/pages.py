@@ -108,22 +108,28 @@ class Compare:
     Raw pages: fp32 values within 1e-5 of the unit's largest; binary16
     values bit-exact except where the GPU's value is the binary16 rounding of
     a value within 4e-6 x max|X| of the unit from X (near a rounding
-    midpoint, or in the subnormal range where the spacing is absolute).  The GPU evaluates X = g x + k u in fp32,
-    whose error is absolute, a few ulps of the largest terms (their
-    magnitude is that of max|X|), and rounds that to binary16, whose spacing
-    at X is 2^-10 |X|: an element flips with probability about
-    2^-10 max|X| / |X|, so the count is bounded by 1e-2 of the values."""
+    midpoint, or in the subnormal range where the spacing is absolute).  The
+    GPU evaluates X (or a pivot row's mu) in fp32, a few ulps off the exact
+    value, and rounds that to binary16, whose rounding midpoints are 2^-10 |X|
+    apart: a value flips with probability of order 2^-12 max|X| / |X|.
+    Measured over every GPU test: 483 of 6.4 M binary16 values (7.6e-5), at
+    most 1.4e-4 in one test; the count is bounded by 3e-4 of the values.
+    Binary16 scale flips: 5 in 626 K rows (8e-6), at most 2 of 4,800 rows in
+    one test; bounded by max(3, 1e-3 x rows)."""
 
     def __init__(self, rtol: float = 1e-5, tie_rel: float = 1e-4, max_tie_frac: float = 1e-4,
-                 scale_flip_rel: float = 1e-5, raw_tie_rel: float = 4e-6, max_raw_tie_frac: float = 1e-2):
+                 scale_flip_rel: float = 1e-5, raw_tie_rel: float = 4e-6, max_raw_tie_frac: float = 3e-4,
+                 max_scale_flip_frac: float = 1e-3):
         self.rtol, self.tie_rel, self.max_tie_frac = rtol, tie_rel, max_tie_frac
         self.scale_flip_rel = scale_flip_rel
         self.raw_tie_rel, self.max_raw_tie_frac = raw_tie_rel, max_raw_tie_frac
+        self.max_scale_flip_frac = max_scale_flip_frac
         self.codes = 0
         self.values = 0
         self.ties = []
         self.flips = []
         self.raw_ties = 0
+        self.raw_flips = []  # (where, row, column, gpu value, oracle value, oracle's fp32 value)
         self.worst_y = 0.0
         self.worst_s = 0.0
         self.worst_x = 0.0
@@ -216,6 +222,9 @@ class Compare:
             assert near.all(), (f"{int((~near).sum())} pivot mismatches beyond the fp32 error window {where}: "
                                 f"gpu {xg[diff][~near][:5]} ref {xr[diff][~near][:5]} mu {x[~near][:5]}")
             self.raw_ties += int(diff.sum())
+            rows = np.nonzero(piv)[0]
+            for (a, b) in zip(*np.nonzero(diff)):
+                self.raw_flips.append((where, int(rows[a]), int(b), float(xg[a, b]), float(xr[a, b]), float(M[a, b])))
 
     def raw(self, page_gpu, page_ref, quot, row_bits, where=""):
         """A raw page: fp32 values within rtol of the unit's largest; binary16
@@ -240,6 +249,8 @@ class Compare:
             assert not bad.any(), (f"{int(bad.sum())} binary16 mismatches beyond the fp32 error window {where}: "
                                    f"gpu {xg[ii, jj][bad][:5]} ref {xr[ii, jj][bad][:5]} X {x[bad][:5]}")
             self.raw_ties += len(ii)
+            for a, b in zip(ii, jj):
+                self.raw_flips.append((where, int(a), int(b), float(xg[a, b]), float(xr[a, b]), float(X[a, b])))
 
     def finish(self):
         frac = len(self.ties) / max(self.codes, 1)
@@ -247,6 +258,8 @@ class Compare:
             print("near-tie:", t)
         for f in self.flips[:10]:
             print("binary16 scale flip:", f)
+        for f in self.raw_flips[:20]:
+            print("binary16 value flip (where, row, col, gpu, oracle, oracle fp32):", f)
         print(f"codes compared {self.codes}, near-ties {len(self.ties)} ({frac:.2e}), "
               f"scale flips {len(self.flips)}, raw values {self.values}, raw ties {self.raw_ties}, "
               f"worst y rel {self.worst_y:.2e}, worst scale rel {self.worst_s:.2e}, "
@@ -255,6 +268,6 @@ class Compare:
               f"with a scale flip not compared)")
         assert frac <= self.max_tie_frac, f"tie fraction {frac:.3g} above {self.max_tie_frac}"
         rows = self.codes // 128
-        assert len(self.flips) <= max(2, 1e-2 * rows), f"{len(self.flips)} scale flips in {rows} rows"
+        assert len(self.flips) <= max(3, self.max_scale_flip_frac * rows), f"{len(self.flips)} scale flips in {rows} rows"
         rfrac = self.raw_ties / max(self.values, 1)
         assert rfrac <= self.max_raw_tie_frac, f"raw tie fraction {rfrac:.3g} above {self.max_raw_tie_frac}"
