@@ -76,14 +76,17 @@ def kernel_sha() -> str:
     return hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()[:16]
 
 
-def recorded_traffic(config: int):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel
-    source is unchanged since it was taken; else None."""
+def recorded_traffic(config: int, requests=None):
+    """DRAM bytes (read + write) per launch from the committed ncu summary, if
+    the kernel source is unchanged since it was taken and the record is of
+    this workload's size; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     d = json.load(open(TRAFFIC_FILE))
     e = d.get(f"config{config}")
     if not e or e.get("kernel_sha") != kernel_sha():
+        return None
+    if "requests" in e and requests is not None and e["requests"] != requests:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -371,7 +374,7 @@ def run_ours(args, rank: int, world: int):
     kernel_s = statistics.mean(times) * 1e-3
     peak, peak_kind = peaks()
     achieved = bytes_per_launch / kernel_s / 1e9
-    traffic = recorded_traffic(args.config)
+    traffic = recorded_traffic(args.config, wl.R)
 
     # ---- end to end through the public API: one pinned host block of inputs in,
     # y out, through stq_decode_step_host_block (its two copies and the decode are

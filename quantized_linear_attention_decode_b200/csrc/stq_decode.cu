@@ -101,6 +101,7 @@ struct __align__(128) Smem {
     float beta[kStages], alpha[kStages];
     uint32_t raw[8][5];  // {req, slot, head offset, page bytes, head} of tile k in raw[k % 8]
     uint32_t flags;
+    uint32_t stop;     // a row-setup wait gave up (set by warps 4-7, read by all after a barrier)
     unsigned long long full[kStages];
     uint8_t *fit_page[2];    // page of the tile whose fit is pending, by tile parity
     uint32_t fit_pending[2];
@@ -202,14 +203,30 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// named CTA barriers (ids 1-15; 0 is __syncthreads): arrive without waiting, or wait
+__device__ __forceinline__ void bar_arrive(int id, int count)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void bar_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void fence_mbar_init()
 {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// packed pair arithmetic (sm_100: one instruction for two fp32 lanes)
+// packed pair arithmetic (sm_100: one instruction for two fp32 lanes).  NV selects the
+// compiler's float2 builtins (its own register pairing and scheduling) over inline PTX;
+// which one the compiler turns into the faster code differs between the kernel's
+// instantiations (measured), so each instantiation picks its own.
+template <bool NV>
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
 {
+    if constexpr (NV) return __ffma2_rn(a, b, c);
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
@@ -219,8 +236,10 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c)
     return d;
 }
 
+template <bool NV>
 __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
 {
+    if constexpr (NV) return __fadd2_rn(a, b);
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -230,8 +249,10 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
     return d;
 }
 
+template <bool NV>
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
 {
+    if constexpr (NV) return __fmul2_rn(a, b);
     float2 d;
     asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
         "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
@@ -294,15 +315,16 @@ template <> struct Codec<8> {
         w.y = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
         *reinterpret_cast<uint2 *>(rowg + cg * 8) = w;
     }
+    template <bool NV>
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
         const uint2 w = *reinterpret_cast<const uint2 *>(rowp + cg * 8);
         const uint32_t x0 = w.x ^ 0x80808080u, x1 = w.y ^ 0x80808080u;
         const float2 off = make_float2(-8388736.0f, -8388736.0f);  // -(2^23 + 128)
-        z[0] = fadd2(make_float2(f_of(__byte_perm(x0, 0x4B000000u, 0x7650)), f_of(__byte_perm(x0, 0x4B000000u, 0x7651))), off);
-        z[1] = fadd2(make_float2(f_of(__byte_perm(x0, 0x4B000000u, 0x7652)), f_of(__byte_perm(x0, 0x4B000000u, 0x7653))), off);
-        z[2] = fadd2(make_float2(f_of(__byte_perm(x1, 0x4B000000u, 0x7650)), f_of(__byte_perm(x1, 0x4B000000u, 0x7651))), off);
-        z[3] = fadd2(make_float2(f_of(__byte_perm(x1, 0x4B000000u, 0x7652)), f_of(__byte_perm(x1, 0x4B000000u, 0x7653))), off);
+        z[0] = fadd2<NV>(make_float2(f_of(__byte_perm(x0, 0x4B000000u, 0x7650)), f_of(__byte_perm(x0, 0x4B000000u, 0x7651))), off);
+        z[1] = fadd2<NV>(make_float2(f_of(__byte_perm(x0, 0x4B000000u, 0x7652)), f_of(__byte_perm(x0, 0x4B000000u, 0x7653))), off);
+        z[2] = fadd2<NV>(make_float2(f_of(__byte_perm(x1, 0x4B000000u, 0x7650)), f_of(__byte_perm(x1, 0x4B000000u, 0x7651))), off);
+        z[3] = fadd2<NV>(make_float2(f_of(__byte_perm(x1, 0x4B000000u, 0x7652)), f_of(__byte_perm(x1, 0x4B000000u, 0x7653))), off);
     }
 };
 
@@ -316,6 +338,7 @@ template <> struct Codec<4> {
         for (int t = 1; t < 8; ++t) acc += b[t] << (4 * t);
         *reinterpret_cast<uint32_t *>(rowg + cg * 4) = (acc - 0xFB000000u) ^ 0x88888888u;
     }
+    template <bool NV>
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
         // code t at bits [4t, 4t + 4); codes 5..7 are shifted down to offsets 0, 4, 8
@@ -329,10 +352,10 @@ template <> struct Codec<4> {
         const uint32_t c5 = masked_field<0xFu, 0x4B000008u>(t);
         const uint32_t c6 = masked_field<0xF0u, 0x49000080u>(t);
         const uint32_t c7 = masked_field<0xF00u, 0x47000800u>(t);
-        z[0] = fadd2(make_float2(f_of(c0), f_of(c1)), make_float2(-8388616.0f, -524296.0f));
-        z[1] = fadd2(make_float2(f_of(c2), f_of(c3)), make_float2(-32776.0f, -2056.0f));
-        z[2] = fadd2(make_float2(f_of(c4), f_of(c5)), make_float2(-136.0f, -8388616.0f));
-        z[3] = fadd2(make_float2(f_of(c6), f_of(c7)), make_float2(-524296.0f, -32776.0f));
+        z[0] = fadd2<NV>(make_float2(f_of(c0), f_of(c1)), make_float2(-8388616.0f, -524296.0f));
+        z[1] = fadd2<NV>(make_float2(f_of(c2), f_of(c3)), make_float2(-32776.0f, -2056.0f));
+        z[2] = fadd2<NV>(make_float2(f_of(c4), f_of(c5)), make_float2(-136.0f, -8388616.0f));
+        z[3] = fadd2<NV>(make_float2(f_of(c6), f_of(c7)), make_float2(-524296.0f, -32776.0f));
     }
 };
 
@@ -350,6 +373,7 @@ template <> struct Codec<6> {
         *reinterpret_cast<uint32_t *>(rowg + cg * 4) = lo;
         *reinterpret_cast<uint16_t *>(rowg + 64 + cg * 2) = static_cast<uint16_t>(hi);
     }
+    template <bool NV>
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
         const uint32_t lo = *reinterpret_cast<const uint32_t *>(rowp + cg * 4);
@@ -364,10 +388,10 @@ template <> struct Codec<6> {
         const uint32_t c5 = masked_field<0x3Fu, 0x4B000020u>(y);
         const uint32_t c6 = masked_field<0xFC0u, 0x48000800u>(y);
         const uint32_t c7 = masked_field<0x3F000u, 0x45020000u>(y);
-        z[0] = fadd2(make_float2(f_of(c0), f_of(c1)), make_float2(-8388640.0f, -131104.0f));
-        z[1] = fadd2(make_float2(f_of(c2), f_of(c3)), make_float2(-2080.0f, -8388640.0f));
-        z[2] = fadd2(make_float2(f_of(c4), f_of(c5)), make_float2(-131104.0f, -8388640.0f));
-        z[3] = fadd2(make_float2(f_of(c6), f_of(c7)), make_float2(-131104.0f, -2080.0f));
+        z[0] = fadd2<NV>(make_float2(f_of(c0), f_of(c1)), make_float2(-8388640.0f, -131104.0f));
+        z[1] = fadd2<NV>(make_float2(f_of(c2), f_of(c3)), make_float2(-2080.0f, -8388640.0f));
+        z[2] = fadd2<NV>(make_float2(f_of(c4), f_of(c5)), make_float2(-131104.0f, -8388640.0f));
+        z[3] = fadd2<NV>(make_float2(f_of(c6), f_of(c7)), make_float2(-131104.0f, -2080.0f));
     }
 };
 
@@ -376,6 +400,7 @@ template <> struct Codec<6> {
 // columns are one 16-byte vector.  The scale slot of the row holds 1, so the
 // row enters both passes like a quantized row whose codes are mu.
 struct Pivot16 {
+    template <bool NV>
     __device__ __forceinline__ static void unpack(const uint8_t *rowp, int cg, float2 z[4])
     {
         const uint4 w = *reinterpret_cast<const uint4 *>(rowp + cg * 16);
@@ -399,12 +424,13 @@ struct Pivot16 {
     }
 };
 
+template <bool NV>
 __device__ __forceinline__ void unpack_any(int b, const uint8_t *rowp, int cg, float2 z[4])
 {
-    if (b == 16) Pivot16::unpack(rowp, cg, z);
-    else if (b == 8) Codec<8>::unpack(rowp, cg, z);
-    else if (b == 6) Codec<6>::unpack(rowp, cg, z);
-    else Codec<4>::unpack(rowp, cg, z);
+    if (b == 16) Pivot16::unpack<NV>(rowp, cg, z);
+    else if (b == 8) Codec<8>::unpack<NV>(rowp, cg, z);
+    else if (b == 6) Codec<6>::unpack<NV>(rowp, cg, z);
+    else Codec<4>::unpack<NV>(rowp, cg, z);
 }
 
 __device__ __forceinline__ void store_any(int b, uint8_t *rowg, int cg, const uint32_t bits[8])
@@ -431,7 +457,7 @@ __device__ __forceinline__ float magic_out(int b)
 // per-warp partials in red.  B = 4, 6, 8: every row has B bits, at
 // 16 B i (GDN) or, with PR, at the row table's offsets (a KDA warp whose
 // rows share one width); B = 0: per-row widths (KDA).
-template <int B, int SB, bool FIT, bool ACC = true, bool PR = false>
+template <int B, int SB, bool FIT, bool NV, bool ACC = true, bool PR = false>
 __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -454,28 +480,28 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
 #pragma unroll
     for (int ii = 0; ii < 8; ++ii) {
         const int i = i0 + ii;
-        if (B != 0 && PR) Codec<B == 0 ? 8 : B>::unpack(S.page + R.off[i], cg, z[ii]);
-        else if (B != 0) Codec<B == 0 ? 8 : B>::unpack(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
-        else unpack_any(R.bits[i], S.page + R.off[i], cg, z[ii]);
+        if (B != 0 && PR) Codec<B == 0 ? 8 : B>::template unpack<NV>(S.page + R.off[i], cg, z[ii]);
+        else if (B != 0) Codec<B == 0 ? 8 : B>::template unpack<NV>(S.page + SB * kD + (FIT ? kFitBytes : 0) + 16 * B * i, cg, z[ii]);
+        else unpack_any<NV>(R.bits[i], S.page + R.off[i], cg, z[ii]);
         if (B == 0 && FIT && R.bits[i] == 16) {
 #pragma unroll
-            for (int p = 0; p < 4; ++p) z[ii][p] = fmul2(z[ii][p], ic[p]);
+            for (int p = 0; p < 4; ++p) z[ii][p] = fmul2<NV>(z[ii][p], ic[p]);
         }
         if constexpr (ACC) {
             const float4 kl = R.kl[i];
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
-                av[p] = ffma2(make_float2(kl.x, kl.y), z[ii][p], av[p]);
-                ay[p] = ffma2(make_float2(kl.z, kl.w), z[ii][p], ay[p]);
+                av[p] = ffma2<NV>(make_float2(kl.x, kl.y), z[ii][p], av[p]);
+                ay[p] = ffma2<NV>(make_float2(kl.z, kl.w), z[ii][p], ay[p]);
             }
         }
     }
     if constexpr (ACC) {
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            av[p] = fadd2(av[p], make_float2(__shfl_xor_sync(0xffffffffu, av[p].x, 16),
+            av[p] = fadd2<NV>(av[p], make_float2(__shfl_xor_sync(0xffffffffu, av[p].x, 16),
                                              __shfl_xor_sync(0xffffffffu, av[p].y, 16)));
-            ay[p] = fadd2(ay[p], make_float2(__shfl_xor_sync(0xffffffffu, ay[p].x, 16),
+            ay[p] = fadd2<NV>(ay[p], make_float2(__shfl_xor_sync(0xffffffffu, ay[p].x, 16),
                                              __shfl_xor_sync(0xffffffffu, ay[p].y, 16)));
         }
         // half 0 keeps the v-sums, half 1 the y-sums; column j of a sum sits at
@@ -603,7 +629,7 @@ __device__ __forceinline__ void row_setup(Smem &sm, const Stage &S, RowCoef &R, 
 // Pass 2: w = z + h u~, row absmax (8 columns per thread, then the 16 column
 // groups of the half-warp through shared memory), new scale, requantise,
 // store codes and scales to the page in global memory.
-template <int B, int SB, bool FIT, bool PR = false>
+template <int B, int SB, bool FIT, bool NV, bool PR = false>
 __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S, float2 z[8][4])
 {
     const int tid = threadIdx.x;
@@ -632,7 +658,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
         for (int ii = 0; ii < 8; ++ii) {
             const float2 h2 = make_float2(hs[ii], hs[ii]);
 #pragma unroll
-            for (int p = 0; p < 4; ++p) z[ii][p] = ffma2(h2, ut2[p], z[ii][p]);
+            for (int p = 0; p < 4; ++p) z[ii][p] = ffma2<NV>(h2, ut2[p], z[ii][p]);
         }
     } else {
 #pragma unroll
@@ -640,10 +666,10 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
             const float2 h2 = make_float2(hs[ii], hs[ii]);
             if (!((deg >> ii) & 1u)) {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) z[ii][p] = ffma2(h2, ut2[p], z[ii][p]);
+                for (int p = 0; p < 4; ++p) z[ii][p] = ffma2<NV>(h2, ut2[p], z[ii][p]);
             } else {
 #pragma unroll
-                for (int p = 0; p < 4; ++p) z[ii][p] = fmul2(h2, ut2[p]);
+                for (int p = 0; p < 4; ++p) z[ii][p] = fmul2<NV>(h2, ut2[p]);
             }
         }
     }
@@ -750,14 +776,14 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
             const float2 m2 = make_float2(R.mrq[i], R.mrq[i]);
             float2 t[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) t[p] = fmul2(z[ii][p], m2);
+            for (int p = 0; p < 4; ++p) t[p] = fmul2<NV>(z[ii][p], m2);
             if (FIT) {
                 const float4 a = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg);
                 const float4 b = *reinterpret_cast<const float4 *>(S.page + SB * kD + 32 * cg + 16);
-                t[0] = fmul2(t[0], make_float2(a.x, a.y));
-                t[1] = fmul2(t[1], make_float2(a.z, a.w));
-                t[2] = fmul2(t[2], make_float2(b.x, b.y));
-                t[3] = fmul2(t[3], make_float2(b.z, b.w));
+                t[0] = fmul2<NV>(t[0], make_float2(a.x, a.y));
+                t[1] = fmul2<NV>(t[1], make_float2(a.z, a.w));
+                t[2] = fmul2<NV>(t[2], make_float2(b.x, b.y));
+                t[3] = fmul2<NV>(t[3], make_float2(b.z, b.w));
             }
             Pivot16::store(page + R.off[i], cg, t);
             continue;
@@ -767,7 +793,7 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
         uint32_t bits[8];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            float2 t = ffma2(z[ii][p], inv2, mg2);
+            float2 t = ffma2<NV>(z[ii][p], inv2, mg2);
             if (SB == 2 && ((clipm >> ii) & 1u)) {
                 // the binary16 scale rounded below a / q_b by up to half a subnormal step:
                 // clip the rounded quotient to [-q_b, q_b]
@@ -779,10 +805,10 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
             bits[2 * p + 1] = __float_as_uint(t.y);
             if (FIT) {
                 // z' = t - mg exactly (the new code); A z' w and B z'^2 into the column sums
-                const float2 zq = fadd2(t, make_float2(-mg, -mg));
+                const float2 zq = fadd2<NV>(t, make_float2(-mg, -mg));
                 const float A = sm.rowA[i], Bc = sm.rowB[i];
-                fnum[p] = ffma2(make_float2(A, A), fmul2(zq, z[ii][p]), fnum[p]);
-                fden[p] = ffma2(make_float2(Bc, Bc), fmul2(zq, zq), fden[p]);
+                fnum[p] = ffma2<NV>(make_float2(A, A), fmul2<NV>(zq, z[ii][p]), fnum[p]);
+                fden[p] = ffma2<NV>(make_float2(Bc, Bc), fmul2<NV>(zq, zq), fden[p]);
             }
         }
         if (B != 0 && PR) Codec<B == 0 ? 8 : B>::store(page + R.off[i], cg, bits);
@@ -793,9 +819,9 @@ __device__ __forceinline__ void pass2(Smem &sm, const RowCoef &R, const Stage &S
         // per-warp partials, laid out as pass 1's column sums (half 0 numerators, half 1 denominators)
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            fnum[p] = fadd2(fnum[p], make_float2(__shfl_xor_sync(0xffffffffu, fnum[p].x, 16),
+            fnum[p] = fadd2<NV>(fnum[p], make_float2(__shfl_xor_sync(0xffffffffu, fnum[p].x, 16),
                                                  __shfl_xor_sync(0xffffffffu, fnum[p].y, 16)));
-            fden[p] = fadd2(fden[p], make_float2(__shfl_xor_sync(0xffffffffu, fden[p].x, 16),
+            fden[p] = fadd2<NV>(fden[p], make_float2(__shfl_xor_sync(0xffffffffu, fden[p].x, 16),
                                                  __shfl_xor_sync(0xffffffffu, fden[p].y, 16)));
         }
         const float2 *src = rgl == 0 ? fnum : fden;
@@ -921,15 +947,18 @@ __device__ __forceinline__ TileRaw raw_from_smem(const Smem &sm, int k)
 
 // Persistent CTA: tiles first, first + G, first + 2G, ... (G = gridDim.x).
 // Per tile i (stage i % 4, row data rc[i % 2]):
-//   all:       pass 1 of tile i                                        | barrier
+//   all:       pass 1 of tile i                                        | __syncthreads
 //   thread 96: issue tile i + 3 (page and head block) into the stage of tile i - 1
 //   all:       cp.async prefetch of tile i + 3's vectors, tile i + 5's location
-//   warps 0-3: column epilogue of tile i (y, u / c)
-//   warps 4-7: wait for tile i + 1's stage, its row coefficients       | barrier
+//   warps 0-3: column epilogue of tile i (y, u / c)   | arrive 1, sync 2 (warps 0-3)
+//   warps 4-7: wait for tile i + 1's stage, its row coefficients   | arrive 3, sync 1
 //   all:       pass 2 of tile i (codes held in registers; new codes and scales to global memory)
-// A stage is last read before the second barrier of its tile (pass 2 reads
-// only registers and the row data); thread 96 refills it after the first
-// barrier of the next tile.
+//   warps 0-3: sync 3 (tile i + 1's row data is in) before their next pass 1
+// Named barriers let warps 0-3 start pass 2 as soon as the four epilogue warps
+// are done, without waiting for warps 4-7's row setup of the next tile.  A
+// stage is last read before barrier 1 of its tile (pass 2 reads only registers,
+// the row data and, for fitted pivot rows, the column factors before the next
+// __syncthreads); thread 96 refills it after the first barrier of the next tile.
 template <int KIND, int SB, int MODE, bool FIT>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeIO io, int tiles)
 {
@@ -942,6 +971,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
 
     if (tid == 0) {
         sm.flags = 0;
+        sm.stop = 0;
         sm.fit_pending[0] = sm.fit_pending[1] = 0;
         for (int s = 0; s < kStages; ++s) mbar_init(&sm.full[s], 1);
         fence_mbar_init();
@@ -988,18 +1018,19 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         const int b = valid ? R.bits[0] : 8;
         float2 z[8][4];
         constexpr bool kAcc = MODE != kWriteback;
+        constexpr bool kNV = KIND == STQ_GDN && !FIT;  // the builtins measure faster only here
         if (valid) {
             if constexpr (KIND == STQ_KDA) {
                 // per-row widths (and KDA pivot rows), or the one width of this warp's rows
                 const int wb = R.wbits[tid >> 5];
-                if (wb == 6) pass1<6, SB, FIT, kAcc, true>(sm, S, R, z);
-                else if (wb == 8) pass1<8, SB, FIT, kAcc, true>(sm, S, R, z);
-                else if (wb == 4) pass1<4, SB, FIT, kAcc, true>(sm, S, R, z);
-                else pass1<0, SB, FIT, kAcc>(sm, S, R, z);
+                if (wb == 6) pass1<6, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
+                else if (wb == 8) pass1<8, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
+                else if (wb == 4) pass1<4, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
+                else pass1<0, SB, FIT, kNV, kAcc>(sm, S, R, z);
             }
-            else if (b == 8) pass1<8, SB, FIT, kAcc>(sm, S, R, z);
-            else if (b == 6) pass1<6, SB, FIT, kAcc>(sm, S, R, z);
-            else pass1<4, SB, FIT, kAcc>(sm, S, R, z);
+            else if (b == 8) pass1<8, SB, FIT, kNV, kAcc>(sm, S, R, z);
+            else if (b == 6) pass1<6, SB, FIT, kNV, kAcc>(sm, S, R, z);
+            else pass1<4, SB, FIT, kNV, kAcc>(sm, S, R, z);
         }
         cp_async_wait<1>();
         __syncthreads();
@@ -1012,7 +1043,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
             h5 -= p.H;
             ++n5;
         }
-        bool tout = false;
+        // barrier 1: u~ of this tile ready (warps 0-3 arrive, warps 4-7 wait); barrier 2: among
+        // warps 0-3, every epilogue read of the partial sums done; barrier 3: the next tile's
+        // row data ready (warps 4-7 arrive, warps 0-3 wait before their next pass 1)
         if (tid < kD) {
             constexpr bool kFits = FIT && MODE != kReadout;
             if (kFits) fit_finish<SB>(sm, (i + 1) & 1);  // the previous tile's factors
@@ -1021,25 +1054,35 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
                 sm.fit_page[i & 1] = R.page;
                 sm.fit_pending[i & 1] = valid;
             }
-        } else if (tile + G < tiles) {
-            const int sn = (i + 1) % kStages;
-            if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1, p.wait_ns)))
-                row_setup<KIND, SB, MODE, FIT>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
-            else
-                tout = true;
+            bar_arrive(1, kThreads);
+            bar_sync(2, kD);
+        } else {
+            if (tile + G < tiles) {
+                const int sn = (i + 1) % kStages;
+                if (__all_sync(0xffffffffu, mbar_wait_bounded(&sm.full[sn], ((i + 1) / kStages) & 1, p.wait_ns)))
+                    row_setup<KIND, SB, MODE, FIT>(sm, sm.st[sn], sm.rc[(i + 1) & 1], sn);
+                else if ((tid & 31) == 0)
+                    sm.stop = 1;
+            }
+            bar_arrive(3, kThreads);
+            bar_sync(1, kThreads);
+            timed_out = sm.stop != 0;
         }
-        timed_out = __syncthreads_or(tout) != 0;
         if (valid && MODE != kReadout) {
             if constexpr (KIND == STQ_KDA) {
                 const int wb = R.wbits[tid >> 5];
-                if (wb == 6) pass2<6, SB, FIT, true>(sm, R, S, z);
-                else if (wb == 8) pass2<8, SB, FIT, true>(sm, R, S, z);
-                else if (wb == 4) pass2<4, SB, FIT, true>(sm, R, S, z);
-                else pass2<0, SB, FIT>(sm, R, S, z);
+                if (wb == 6) pass2<6, SB, FIT, kNV, true>(sm, R, S, z);
+                else if (wb == 8) pass2<8, SB, FIT, kNV, true>(sm, R, S, z);
+                else if (wb == 4) pass2<4, SB, FIT, kNV, true>(sm, R, S, z);
+                else pass2<0, SB, FIT, kNV>(sm, R, S, z);
             }
-            else if (b == 8) pass2<8, SB, FIT>(sm, R, S, z);
-            else if (b == 6) pass2<6, SB, FIT>(sm, R, S, z);
-            else pass2<4, SB, FIT>(sm, R, S, z);
+            else if (b == 8) pass2<8, SB, FIT, kNV>(sm, R, S, z);
+            else if (b == 6) pass2<6, SB, FIT, kNV>(sm, R, S, z);
+            else pass2<4, SB, FIT, kNV>(sm, R, S, z);
+        }
+        if (tid < kD) {
+            bar_sync(3, kThreads);
+            timed_out = sm.stop != 0;
         }
     }
     if (FIT && MODE != kReadout) {
