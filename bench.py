@@ -429,6 +429,10 @@ def run_ours(args, rank: int, world: int):
     if rank == 0 and world == 1 and not args.no_sweep:
         with torch.cuda.nvtx.range("bench: pool sweep"):
             sweep = pool_sweep(stq, flush, stream, peak)
+    kda = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        with torch.cuda.nvtx.range("bench: KDA variants"):
+            kda = kda_variants(stq, flush, stream, peak)
     loop = None
     if rank == 0 and world == 1 and not args.no_layer_loop:
         with torch.cuda.nvtx.range("bench: layer loop"):
@@ -468,6 +472,7 @@ def run_ours(args, rank: int, world: int):
         "gpu_launches": launches,
         "clocks": sampler.summary(),
         "pool_sweep": sweep,
+        "kda_variants": kda,
         "layer_loop": loop,
         "drift": drift_log,
     }
@@ -543,6 +548,66 @@ def pool_sweep(stq, flush, stream, peak, reps: int = 20):
         out.append(row)
         del x, y
         torch.cuda.empty_cache()
+    return out
+
+
+def kda_allocated_bits(stq, H: int, seed: int, pivots: int = 8):
+    """Per-row widths of H KDA heads from the lifetime-aware allocator: a 6-bit budget
+    over {4, 6, 8} per head (Lagrangian) on synthetic calibration statistics (row
+    distortion d_u(b) ~ logU(e^-2, e^2) 4^-k, mean log retention of U(0.8, 0.9995) decays,
+    horizon 8192), then the head's `pivots` riskiest rows kept as FP16 pivots."""
+    out = []
+    for h in range(H):
+        d0 = synth.log_uniform(synth.stream_key(seed, 90, 1, h), 128, np.exp(-2.0), np.exp(2.0))
+        dist = d0[:, None] * 4.0 ** (-np.arange(3)[None, :])
+        keep = 0.8 + (0.9995 - 0.8) * synth.uniform(synth.stream_key(seed, 90, 2, h), 128)
+        w = stq.stq_lifetime_weight(np.log(keep), 8192)
+        bits, _ = stq.stq_allocate_bits(np.full(128, 128.0), [4, 6, 8], dist, w, 6.0,
+                                        method=stq.STQ_ALLOC_LAGRANGE, num_pivots=pivots, pivot_bits=16)
+        out.append(bits)
+    return np.concatenate(out)
+
+
+def kda_variants(stq, flush, stream, peak, reps: int = 20):
+    """KDA 128 requests x 32 heads, one token per launch (median over `reps`
+    launches, L2 flushed before each, from the zero state after 3 warm-up steps):
+    the workload's 32/64/32 rows per head at 4/6/8 bits; widths from the
+    lifetime-aware allocator with 8 FP16 pivot rows per head; and those widths
+    with column factors refitted every step (the page's KDA setting: pivot
+    rows, fit over the non-pivot rows)."""
+    import dataclasses
+    import torch
+    wl = synth.make_workload(3)
+    alloc = kda_allocated_bits(stq, wl.H, 0)
+    rw = synth.log_uniform(synth.stream_key(0, 90, 3), wl.H * 128, 0.5, 2.0).astype(np.float32)
+    req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
+    slot = torch.zeros(wl.R, dtype=torch.int32, device="cuda")
+    x = {k: torch.from_numpy(v).cuda() for k, v in wl.step_inputs(0).items()}
+    y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
+    out = {"requests": wl.R, "heads": wl.H, "mean_bits_allocated": float(alloc.astype(np.float64).mean())}
+    for tag, bits, flags in (("rows_32_64_32", wl.unit_bits, 0), ("allocated_pivots", alloc, 0),
+                             ("allocated_pivots_fit", alloc, stq.STQ_FIT_COLUMNS)):
+        pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, bits, wl.row_factor, wl.col_factor,
+                                   flags=flags, row_weight=rw if flags else None)
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
+            b.record(stream)
+            if i >= 3:
+                ts.append((a, b))
+        torch.cuda.synchronize()
+        stq.stq_pool_check(pool, stream)
+        med = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e-3
+        nbytes, _ = workload_info(dataclasses.replace(wl, unit_bits=np.asarray(bits)))
+        if flags:
+            nbytes += wl.R * wl.H * 2 * 512  # the page's own column factors, read and written
+        out[tag] = {"kernel_us": med * 1e6, "head_steps_per_s": wl.R * wl.H / med,
+                    "gbs": nbytes / med / 1e9, "frac": nbytes / med / 1e9 / peak}
+        pool.close()
+    torch.cuda.empty_cache()
     return out
 
 
