@@ -79,9 +79,12 @@ typedef struct stq_pool stq_pool;
  * offline step (3): the riskiest units are kept in FP16, 32 of 2304 GDN heads
  * and 512 of 81920 KDA rows in the page's setting).  A pivot row keeps its
  * scale slot, which holds 1, and stores mu_ij = X_ij / (r_i c_j) rounded once
- * to binary16 (the state itself when r = c = 1).  A KDA head's page must stay
- * within 16896 bytes (pivot rows averaging at most 8 bits per row over the
- * head), else STQ_ERR_UNSUPPORTED.
+ * to binary16 (the state itself when r = c = 1; X_ij / r_i with
+ * STQ_FIT_COLUMNS).  A KDA head's page (its scales, a fitted page's 512 bytes
+ * of column factors, 16 b_i bytes per row with pivot rows at b = 16, padded
+ * to 128 bytes) must fit the decode kernel's 17408-byte staging buffer: with
+ * fp32 scales, rows averaging at most 8.25 bits (8 when fitted); else
+ * STQ_ERR_UNSUPPORTED.
  * Raw pools hold the state values themselves: every unit at 16 (IEEE
  * binary16, no scales, r and c unused) or every unit at 32 (fp32, the
  * unquantized control the page's state-update timings compare against); fp32
@@ -92,9 +95,13 @@ typedef struct stq_pool stq_pool;
  * quantisation ("core method" dual-axis fit; "method steps", steps 4-5):
  * the codes are taken with the page's current factors, then
  *   c_j <- sum_i w_i^2 v_ij X_ij / sum_i w_i^2 v_ij^2,  v_ij = s_i r_i z_ij,
- * over the head's rows with the frozen row weights w_i (row_weight); a column
+ * over the head's non-pivot rows ("core innovation": c_j is fitted "across
+ * non-pivot rows") with the frozen row weights w_i (row_weight); a column
  * whose codes are all zero keeps its factor.  col_factor gives the factors
- * the first quantisation starts from.  Not with pivot or raw units. */
+ * the first quantisation starts from.  An FP16 pivot row of a fitted page
+ * stores mu_ij = X_ij / r_i (no column factor, so that refitting does not
+ * move it) and reconstructs as r_i mu_ij; a GDN pivot head's page keeps an
+ * unused factor section.  Not with raw pools. */
 #define STQ_FIT_COLUMNS 2u
 
 typedef struct {

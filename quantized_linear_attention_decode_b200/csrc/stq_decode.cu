@@ -49,7 +49,7 @@ constexpr int kReadout = 1;    // steps 1-3: y and u~; the page is only read
 constexpr int kWriteback = 2;  // steps 4-7 given u~: requantise and pack in place
 constexpr int kStages = 4;
 constexpr int kRedStride = 288;  // floats per warp in red: 256 column partials, or the padded row-max exchange
-constexpr int kMaxPage = kMaxStagedPage;               // 16896: every row at 8 bits
+constexpr int kMaxPage = kMaxStagedPage;               // 17408: every row at 8 bits, with fitted factors
 
 struct __align__(128) Stage {
     uint8_t page[kMaxPage];
