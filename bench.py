@@ -478,12 +478,24 @@ def run_ours(args, rank: int, world: int):
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": sampler.summary(),
-        "pool_sweep": sweep,
-        "kda_variants": kda,
-        "layer_loop": loop,
-        "drift": drift_log,
+        # the supplementary records, rounded, the steady-state serving-pool sweep last
+        "drift": compact(drift_log),
+        "layer_loop": compact(loop),
+        "kda_variants": compact(kda),
+        "pool_sweep": compact(sweep),
     }
     print(json.dumps(line), flush=True)
+
+
+def compact(obj, digits: int = 4):
+    """obj with every float rounded to `digits` significant digits (short JSON)."""
+    if isinstance(obj, float):
+        return float(f"{obj:.{digits}g}")
+    if isinstance(obj, dict):
+        return {k: compact(v, digits) for k, v in obj.items()}
+    if isinstance(obj, list):
+        return [compact(v, digits) for v in obj]
+    return obj
 
 
 def copy_rates(torch, host_in, host_out, stream, reps: int = 20):
