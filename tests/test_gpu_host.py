@@ -170,10 +170,11 @@ def _block(pool, n, req, slot, x, pinned=True):
     return blk
 
 
-@pytest.mark.parametrize("config", [2, 3])
-def test_host_block_decode_matches_device_step(config):
+@pytest.mark.parametrize("config, pinned", [(2, True), (3, True), (2, False)])
+def test_host_block_decode_matches_device_step(config, pinned):
     """The single-copy host block: GDN (per-head gate) and KDA (per-row gate)
-    layouts, a subset of requests, three tokens; y and pages bit for bit."""
+    layouts, a subset of requests, three tokens, page-locked and pageable host
+    memory; y and pages bit for bit."""
     wl = synth.make_workload(config, R=24)
     ref, got = _pool(wl), _pool(wl)
     offs, nbytes = stq.stq_host_block_layout(got, 0)
@@ -187,10 +188,11 @@ def test_host_block_decode_matches_device_step(config):
         x = {key: np.ascontiguousarray(inp[key][sel]) for key in KEYS}
         y_ref = torch.empty((n, wl.H, 128), dtype=torch.float32, device="cuda")
         stq.stq_decode_step(ref, _cuda(req), _cuda(slot), *[_cuda(x[key]) for key in KEYS], y_ref)
-        blk = _block(got, n, req, slot, x)
+        blk = _block(got, n, req, slot, x, pinned)
         offs, nbytes = stq.stq_host_block_layout(got, n)
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs) and blk.numel() == nbytes
-        y_got = torch.full((n, wl.H, 128), float("nan")).pin_memory()
+        y_got = torch.full((n, wl.H, 128), float("nan"))
+        y_got = y_got.pin_memory() if pinned else y_got
         stq.stq_decode_step_host_block(got, n, blk, y_got)
         torch.cuda.current_stream().synchronize()
         stq.stq_pool_check(ref)
