@@ -279,11 +279,15 @@ stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const 
  * alignment rule).  On `stream`, after the work already queued there, the
  * library copies the inputs into a device staging buffer that the pool owns,
  * runs the step (the same kernels, so the results are those of
- * stq_decode_step bit for bit) and copies y back; y may be read once
- * `stream` is synchronized.
+ * stq_decode_step bit for bit) and delivers y; y may be read once `stream` is
+ * synchronized.
  *   - Page-locked host memory (cudaHostAlloc, cudaHostRegister) makes the
  *     copies asynchronous; pageable memory works, with copies that block the
  *     host.
+ *   - A page-locked y that the device can address (every page-locked
+ *     allocation on a system with unified addressing) is written by the
+ *     decode kernels directly, across the bus, with no copy back; any other y
+ *     is written to the staging buffer and copied back.
  *   - The inputs must stay unchanged, and y unread, until `stream` has
  *     passed the step.
  *   - The first call, and any call with more entries than every earlier
@@ -315,10 +319,11 @@ stq_status stq_decode_step_host(stq_pool *pool, const int32_t *req_idx, const in
  * from `block` (host memory of at least `bytes` bytes, as laid out above for
  * this n; `bytes` must equal the layout's size, else STQ_ERR_ARG) and y
  * written to the host array y (fp32 [n][H][128]).  One host-to-device copy
- * of the block, the step, one device-to-host copy of y, all on `stream`;
- * the results equal stq_decode_step's bit for bit, and the staging rules
- * (shared buffer, first-call allocation, page-locked memory for
- * asynchronous copies) are those of stq_decode_step_host.
+ * of the block and the step, all on `stream`, with y delivered as by
+ * stq_decode_step_host (written by the kernels when page-locked, else one
+ * device-to-host copy); the results equal stq_decode_step's bit for bit, and
+ * the staging rules (shared buffer, first-call allocation, page-locked memory
+ * for asynchronous copies) are those of stq_decode_step_host.
  */
 stq_status stq_host_block_layout(const stq_pool *pool, int32_t n, size_t offsets[7], size_t *bytes);
 stq_status stq_decode_step_host_block(stq_pool *pool, int32_t n, const void *block, size_t bytes, float *y,

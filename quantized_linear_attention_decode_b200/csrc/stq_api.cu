@@ -739,10 +739,12 @@ stq_status stq_decode_step_static(stq_pool *p, const int32_t *req_idx, const int
 
 // ---------------------------------------------------------------- decode from host buffers
 //
-// Inputs in, one decode, y out, all on the caller's stream.  Cutting the
-// entries into chunks pipelined over separate copy streams measured slower at
-// 2048 tiles (each cross-stream wait costs more than the overlap it buys) and
-// no faster at 8192, so the step stays on one stream.
+// Inputs in, one decode, y out, all on the caller's stream.  A page-locked y
+// is written by the decode kernels themselves across the bus (each warp stores
+// whole 128-byte lines), so it needs no copy back; a pageable y is staged and
+// copied.  Cutting the entries into chunks pipelined over separate copy streams
+// measured slower at 2048 tiles (each cross-stream wait costs more than the
+// overlap it buys) and no faster at 8192, so the step stays on one stream.
 
 }  // extern "C"
 
@@ -800,19 +802,32 @@ cudaError_t host_staging(stq_pool *p, size_t bytes, cudaStream_t stream)
 }
 
 // The step on inputs already copied into the staging buffer (queued on s0),
-// then y copied back to the host; records the pool's staging event.
+// with y written straight to a page-locked y or else copied back to the host;
+// records the pool's staging event.
 stq_status host_decode_and_copy_out(stq_pool *p, int32_t n, const HostLayout &L, float *y, cudaStream_t s0)
 {
     uint8_t *d = p->h_stage;
     const size_t vec = (size_t)n * p->H * kD * sizeof(float);
+    // page-locked y (device-addressable): the kernels write it directly, no copy back
+    float *yk = reinterpret_cast<float *>(d + L.y);
+    bool direct = false;
+    cudaPointerAttributes pa;
+    if (cudaPointerGetAttributes(&pa, y) == cudaSuccess) {
+        if (pa.type == cudaMemoryTypeHost && pa.devicePointer != nullptr) {
+            yk = static_cast<float *>(pa.devicePointer);
+            direct = true;
+        }
+    } else {
+        cudaGetLastError();
+    }
     const stq::DecodeIO io{reinterpret_cast<const int32_t *>(d + L.req), reinterpret_cast<const int32_t *>(d + L.slot),
                            n, reinterpret_cast<const float *>(d + L.q), reinterpret_cast<const float *>(d + L.k),
                            reinterpret_cast<const float *>(d + L.v), reinterpret_cast<const float *>(d + L.beta),
-                           reinterpret_cast<const float *>(d + L.gate), reinterpret_cast<float *>(d + L.y), nullptr};
+                           reinterpret_cast<const float *>(d + L.gate), yk, nullptr};
     cudaError_t e = debug_checks(p, io.req_idx, io.slot_idx, n, s0);
     if (e == cudaSuccess) e = p->raw_bits ? stq::launch_decode_raw(view(p), io, s0) : stq::launch_decode(view(p), io, s0);
     if (e == cudaSuccess && p->pivot_heads) e = stq::launch_decode_pivot_heads(view(p), io, s0);
-    const cudaError_t eo = e == cudaSuccess ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
+    const cudaError_t eo = e == cudaSuccess && !direct ? cudaMemcpyAsync(y, d + L.y, vec, cudaMemcpyDeviceToHost, s0) : e;
     const cudaError_t er = cudaEventRecord(p->h_done, s0);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     if (eo != cudaSuccess) return cuda_fail(eo, "host-decode output copy");

@@ -513,14 +513,11 @@ __device__ __forceinline__ void pass1(Smem &sm, const Stage &S, const RowCoef &R
     }
 }
 
-// Column handled by epilogue thread t (0..127): a permutation under which the
-// 32 lanes of a warp read 32 distinct banks of the column partial sums (whose
-// column j sits at ((j >> 2) & 1) * 64 + (j >> 3) * 4 + (j & 3)).
-__device__ __forceinline__ int epilogue_column(int t)
-{
-    const int w = t >> 5, lane = t & 31;
-    return ((((w >> 1) << 3) + (lane >> 2)) << 3) | ((w & 1) << 2) | (lane & 3);
-}
+// Column handled by epilogue thread t (0..127): column t, so that a warp's y
+// stores are one contiguous 128-byte line (whole lines also when y is page-locked
+// host memory written across the bus); its reads of the partial sums meet 2-way
+// bank conflicts, which measured cheaper than scattered y stores.
+__device__ __forceinline__ int epilogue_column(int t) { return t; }
 
 // Per column (threads 0..127), one tile after pass 2 wrote its partial sums:
 // the refitted factor c_j <- c_j sum_i A_i z'_ij w_ij / sum_i B_i z'_ij^2
