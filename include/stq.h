@@ -287,7 +287,9 @@ stq_status stq_decode_step_static(stq_pool *pool, const int32_t *req_idx, const 
  *   - A page-locked y that the device can address (every page-locked
  *     allocation on a system with unified addressing) is written by the
  *     decode kernels directly, across the bus, with no copy back; any other y
- *     is written to the staging buffer and copied back.
+ *     is written to the staging buffer and copied back.  A page-locked y must
+ *     therefore be writable by the device: memory registered with
+ *     cudaHostRegisterReadOnly is not a valid y.
  *   - The inputs must stay unchanged, and y unread, until `stream` has
  *     passed the step.
  *   - The first call, and any call with more entries than every earlier
