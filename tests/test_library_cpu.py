@@ -212,3 +212,64 @@ def test_compare_checks_binary16_pages():
     bad[256] ^= 0x3  # code 0 of row 0 changes by more than one step
     with pytest.raises(AssertionError):
         Compare().page(bad, page, quot, bits, fmt=1)
+
+
+C_PROGRAM = r"""
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+#include "stq.h"
+
+int main(void)
+{
+    /* pool accounting without a device: 2 requests x 1 slot x 3 GDN heads at 6 bits */
+    const uint8_t bits[3] = {6, 6, 6};
+    stq_pool_desc d;
+    memset(&d, 0, sizeof d);
+    d.kind = STQ_GDN;
+    d.num_requests = 2;
+    d.num_slots = 1;
+    d.num_heads = 3;
+    d.d_k = 128;
+    d.d_v = 128;
+    d.unit_bits = bits;
+    size_t packed = 0, slot = 0;
+    if (stq_desc_bytes(&d, &packed, &slot) != STQ_OK) return 1;
+    if (slot != 3u * (512u + 2048u * 6u) || packed != 2u * slot) return 2;
+    /* a bad description is refused with a message, an unsupported head size with its own status */
+    d.num_requests = 0;
+    if (stq_desc_bytes(&d, &packed, &slot) != STQ_ERR_ARG || strlen(stq_last_error()) == 0) return 3;
+    d.num_requests = 2;
+    d.d_k = 64;
+    if (stq_desc_bytes(&d, &packed, &slot) != STQ_ERR_UNSUPPORTED) return 6;
+    /* L_u for l_u = log(1/2) over 4 steps: 1 + 1/4 + 1/16 + 1/64 */
+    const double l = log(0.5);
+    double w = 0.0;
+    if (stq_lifetime_weight(1, &l, 4, &w) != STQ_OK || fabs(w - 1.328125) > 1e-15) return 4;
+    if (stq_launch_count() != 0) return 5;
+    printf("%s\n", stq_status_str(STQ_OK));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_the_library_links_from_c(tmp_path):
+    """include/stq.h compiles as strict C99 and a C program links against
+    libstq.so and calls its host-side entry points (no device needed)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    stq.load()
+    libdir = os.path.dirname(stq.LIB_PATH)
+    src = tmp_path / "t.c"
+    src.write_text(C_PROGRAM)
+    exe = tmp_path / "t"
+    r = subprocess.run([gcc, "-std=c99", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", libdir, "-lstq", "-lm", "-Wl,-rpath," + libdir],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "STQ_OK", (r.returncode, r.stdout, r.stderr)
