@@ -321,7 +321,9 @@ def run_ours(args, rank: int, world: int):
     dev = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(dev)
     dist = None
-    if world > 1:
+    # under torchrun (LOCAL_WORLD_SIZE set) the process group is used even by a single rank,
+    # so that a one-GPU launch runs the same collective path as the scaling runs
+    if world > 1 or "LOCAL_WORLD_SIZE" in os.environ:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
