@@ -278,7 +278,8 @@ def stq_host_block_layout(pool: Pool, n: int):
 
 def stq_decode_step_host_block(pool: Pool, n: int, block, y, stream=None) -> None:
     """stq_decode_step_host with every input in one host block (a uint8 CPU
-    tensor laid out by stq_host_block_layout): one copy in, one copy of y out."""
+    tensor laid out by stq_host_block_layout): one copy in; a pinned y is written by the
+    kernels directly, any other y is copied back."""
     import torch
     if not isinstance(block, torch.Tensor) or block.device.type != "cpu" or block.dtype != torch.uint8 \
             or not block.is_contiguous():
