@@ -206,3 +206,32 @@ def test_host_block_decode_matches_device_step(config, pinned):
     assert e.value.status == stq.STQ_ERR_ARG
     ref.close()
     got.close()
+
+
+@pytest.mark.parametrize("config", [2, 3])
+def test_host_block_writes_a_pinned_y_in_place_at_an_offset(config):
+    """A page-locked y that starts inside a larger page-locked buffer (an interior
+    pointer, 128 bytes in): the kernels write exactly its n x H x 128 values across
+    the bus and leave the bytes around it alone; the values equal those of the
+    same step with a pageable y (staged and copied back) bit for bit."""
+    wl = synth.make_workload(config, R=12)
+    ref, got = _pool(wl), _pool(wl)
+    n = wl.R
+    inp = wl.step_inputs(0)
+    req = np.arange(n, dtype=np.int32)
+    slot = wl.slot_of_request.astype(np.int32)
+    x = {key: np.ascontiguousarray(inp[key]) for key in KEYS}
+    m = n * wl.H * 128
+    y_ref = torch.full((n, wl.H, 128), float("nan"))  # pageable
+    stq.stq_decode_step_host_block(ref, n, _block(ref, n, req, slot, x), y_ref)
+    big = torch.full((m + 96,), -7.0).pin_memory()
+    y_got = big[32:32 + m].view(n, wl.H, 128)
+    stq.stq_decode_step_host_block(got, n, _block(got, n, req, slot, x), y_got)
+    torch.cuda.current_stream().synchronize()
+    stq.stq_pool_check(ref)
+    stq.stq_pool_check(got)
+    np.testing.assert_array_equal(y_got.numpy(), y_ref.numpy())
+    assert bool((big[:32] == -7.0).all()) and bool((big[32 + m:] == -7.0).all())
+    _same_slots(_slots(ref, wl), _slots(got, wl))
+    ref.close()
+    got.close()
