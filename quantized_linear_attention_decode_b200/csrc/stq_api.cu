@@ -22,6 +22,7 @@ struct stq_pool {
     bool pivots = false;       // FP16 pivot units among quantized ones
     bool pivot_heads = false;  // GDN pivot heads (their own kernel)
     bool fit = false;          // per-page column factors refitted at every quantisation
+    bool per_row = false;      // KDA: every tile on the decode kernel's per-row path
     int device = 0;
     size_t slot_bytes = 0, packed_bytes = 0;
     uint8_t *d_pages = nullptr;
@@ -190,6 +191,7 @@ stq::PoolView view(stq_pool *p)
     v.raw_bits = p->raw_bits;
     v.pivots = p->pivots ? 1 : 0;
     v.fit = p->fit ? 1 : 0;
+    v.per_row = p->per_row ? 1 : 0;
     v.t = p->t;
     v.err = p->d_err;
     // STQ_FAULT=timeout: a wait that nothing completes, given a short limit
@@ -412,6 +414,13 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
             for (int w = 0; w < 8; ++w)
                 for (int g = 0; g < 2; ++g)
                     for (int t = 0; t < 8; ++t) perm[(2 * w + g) * 8 + t] = (uint8_t)order[16 * w + 2 * t + g];
+            // a pass warp takes positions [16 w, 16 w + 16): the width-specialised passes need
+            // one width of 4, 6 or 8 bits there; otherwise the whole pool takes the per-row path
+            // (a launch mixing both kinds of pass measured slower than the per-row path alone)
+            for (int w = 0; w < 8; ++w) {
+                const int lo = hb[order[16 * w]], hi = hb[order[16 * w + 15]];
+                if (lo != hi || lo > 8) p->per_row = true;
+            }
         } else {
             for (int i = 0; i < kD; ++i) perm[i] = (uint8_t)i;
         }

@@ -1018,8 +1018,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         constexpr bool kNV = KIND == STQ_GDN && !FIT;  // the builtins measure faster only here
         if (valid) {
             if constexpr (KIND == STQ_KDA) {
-                // per-row widths (and KDA pivot rows), or the one width of this warp's rows
-                const int wb = R.wbits[tid >> 5];
+                // the one width of this warp's rows, or the per-row path (per-row widths and
+                // pivot rows; the whole pool takes it when any of its tiles needs it)
+                const int wb = p.per_row ? 0 : R.wbits[tid >> 5];
                 if (wb == 6) pass1<6, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
                 else if (wb == 8) pass1<8, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
                 else if (wb == 4) pass1<4, SB, FIT, kNV, kAcc, true>(sm, S, R, z);
@@ -1067,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(PoolView p, DecodeI
         }
         if (valid && MODE != kReadout) {
             if constexpr (KIND == STQ_KDA) {
-                const int wb = R.wbits[tid >> 5];
+                const int wb = p.per_row ? 0 : R.wbits[tid >> 5];
                 if (wb == 6) pass2<6, SB, FIT, kNV, true>(sm, R, S, z);
                 else if (wb == 8) pass2<8, SB, FIT, kNV, true>(sm, R, S, z);
                 else if (wb == 4) pass2<4, SB, FIT, kNV, true>(sm, R, S, z);

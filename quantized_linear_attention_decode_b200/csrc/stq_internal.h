@@ -54,6 +54,8 @@ struct PoolView {
     int raw_bits;        // 16 or 32 in a raw pool (every unit), else 0
     int pivots;          // nonzero if 16-bit (FP16 pivot) units sit among quantized ones
     int fit;             // nonzero: pages carry column factors refitted at every quantisation
+    int per_row;         // KDA: some head has a pass warp whose 16 rows the width-specialised
+                         // passes cannot take, so every tile takes the per-row path
     Tables t;
     uint32_t *err;
     unsigned long long wait_ns;  // limit of every bounded device-side wait
