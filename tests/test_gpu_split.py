@@ -30,11 +30,26 @@ def test_split_teacher_forced_config3_kda():
     _teacher_forced(synth.make_workload(3, R=3, H=4), steps=8, split=True)
 
 
-@pytest.mark.parametrize("config, flags", [(2, 0), (3, 0), (2, stq.STQ_SCALE_F16)])
+def _ragged_kda(R, H, seed=23):
+    """KDA with row widths drawn independently: pass warps mix widths, so the
+    pool runs every tile on the per-row path."""
+    rng = np.random.default_rng(seed)
+    wl = synth.make_workload(3, R=R, H=H)
+    wl.unit_bits = rng.choice(np.array([4, 6, 8], np.uint8), size=H * 128)
+    wl.init = "outlier"
+    return wl
+
+
+def test_split_teacher_forced_kda_per_row_widths():
+    """Split step against the oracle on a KDA pool whose rows take the per-row path."""
+    _teacher_forced(_ragged_kda(3, 4), steps=8, split=True)
+
+
+@pytest.mark.parametrize("config, flags", [(2, 0), (3, 0), (2, stq.STQ_SCALE_F16), ("kda_rows", 0)])
 def test_split_bit_identical_to_fused(config, flags):
     """Same inputs, two pools: the split step's y, codes and scales equal the
-    fused step's bit for bit, every step."""
-    wl = synth.make_workload(config, R=5, H=8)
+    fused step's bit for bit, every step (also on the per-row path)."""
+    wl = _ragged_kda(5, 8) if config == "kda_rows" else synth.make_workload(config, R=5, H=8)
     pools = [stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor,
                                  flags=flags) for _ in range(2)]
     req, slot = _init(wl, pools[0])
