@@ -62,16 +62,21 @@ def test_pivot_quantize_dequantize_bit_exact(config, f16):
     pool.close()
 
 
-def _teacher_forced(wl, steps, f16=False, split=False):
+def _teacher_forced(wl, steps, f16=False, split=False, units=None, check_steps=None):
+    """`steps` decode steps on all requests; `units` ((request, head) pairs, default
+    all) checked against the oracle at `check_steps` (default all)."""
     fmt = (1 if f16 else 0) | PIVOT
     pool, req, slot = _pool(wl, f16)
     rb = wl.row_bits()
     r, c = wl.row_factor.reshape(wl.H, 128), wl.col_factor.reshape(wl.H, 128)
+    units = [(a, h) for a in range(wl.R) for h in range(wl.H)] if units is None else units
+    reqs = sorted({a for a, _ in units})
     cmp = Compare()
     side = torch.cuda.Stream()
     for t in range(steps):
-        before = [split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb, fmt)
-                  for a in range(wl.R)]
+        check = check_steps is None or t in check_steps
+        before = {a: split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb, fmt)
+                  for a in (reqs if check else [])}
         inp = wl.step_inputs(t)
         x = [_cuda(inp[key]) for key in ("q", "k", "v", "beta", "gate")]
         y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
@@ -81,19 +86,20 @@ def _teacher_forced(wl, steps, f16=False, split=False):
         else:
             stq.stq_decode_step(pool, req, slot, *x, y)
         stq.stq_pool_check(pool)
+        if not check:
+            continue
         y = y.cpu().numpy()
-        for a in range(wl.R):
-            after = split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb, fmt)
-            for h in range(wl.H):
-                g = inp["gate"][a, h]
-                g = np.full(128, g, np.float32) if np.ndim(g) == 0 else g
-                page_ref, y_ref, quot, st = orc.step_unit(rb[h], r[h], c[h], before[a][h], inp["q"][a, h],
-                                                          inp["k"][a, h], inp["v"][a, h], inp["beta"][a, h],
-                                                          g, fmt=fmt)
-                assert st == orc.OK
-                where = f"(t={t}, req={a}, head={h})"
-                cmp.y(y[a, h], y_ref, where)
-                cmp.page(after[h], page_ref, quot, rb[h], where, fmt=fmt)
+        after = {a: split_slot(stq.stq_export_slot(pool, a, int(wl.slot_of_request[a])), rb, fmt) for a in reqs}
+        for a, h in units:
+            g = inp["gate"][a, h]
+            g = np.full(128, g, np.float32) if np.ndim(g) == 0 else g
+            page_ref, y_ref, quot, st = orc.step_unit(rb[h], r[h], c[h], before[a][h], inp["q"][a, h],
+                                                      inp["k"][a, h], inp["v"][a, h], inp["beta"][a, h],
+                                                      g, fmt=fmt)
+            assert st == orc.OK
+            where = f"(t={t}, req={a}, head={h})"
+            cmp.y(y[a, h], y_ref, where)
+            cmp.page(after[a][h], page_ref, quot, rb[h], where, fmt=fmt)
     cmp.finish()
     pool.close()
     return cmp
@@ -135,3 +141,16 @@ def test_allocated_widths_with_pivots_run():
     bits, _ = stq.stq_allocate_bits(np.full(wl.H, 16384.0), [4, 6, 8], d, w, 6.0, num_pivots=2, pivot_bits=16)
     assert int(np.count_nonzero(bits == 16)) == 2
     _teacher_forced(dataclasses.replace(wl, unit_bits=bits, init="outlier"), steps=4)
+
+
+def test_allocated_widths_with_pivot_rows_full_size_sampled():
+    """The page's KDA setting at the benchmark's size: 128 requests x 32 heads, per-row
+    widths from the allocator with 8 FP16 pivot rows per head (every tile on the
+    per-row path), three tokens; sampled units checked against the oracle."""
+    from test_gpu_fit import _kda_allocated_pivots
+    wl = _kda_allocated_pivots(128, 32, 21)
+    rng = np.random.default_rng(21)
+    units = [(int(a), int(h)) for a, h in zip(rng.integers(0, wl.R, 12), rng.integers(0, wl.H, 12))]
+    units += [(wl.R - 1, wl.H - 1), (0, 0)]
+    cmp = _teacher_forced(wl, steps=3, units=units, check_steps={0, 2})
+    assert cmp.values == 2 * len(units) * 8 * 128  # the pivot rows' binary16 values
