@@ -444,6 +444,10 @@ def run_ours(args, rank: int, world: int):
     if rank == 0 and world == 1 and not args.no_sweep:
         with torch.cuda.nvtx.range("bench: KDA variants"):
             kda = kda_variants(stq, flush, stream, peak)
+    gpiv = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        with torch.cuda.nvtx.range("bench: GDN pivot heads"):
+            gpiv = gdn_pivot_heads(stq, flush, stream, peak)
     loop = None
     if rank == 0 and world == 1 and not args.no_layer_loop:
         with torch.cuda.nvtx.range("bench: layer loop"):
@@ -486,6 +490,7 @@ def run_ours(args, rank: int, world: int):
         "drift": compact(drift_log),
         "layer_loop": compact(loop),
         "kda_variants": compact(kda),
+        "gdn_pivot_heads": compact(gpiv),
         "pool_sweep": compact(sweep),
     }
     print(json.dumps(line), flush=True)
@@ -631,6 +636,49 @@ def kda_variants(stq, flush, stream, peak, reps: int = 20):
                     "gbs": nbytes / med / 1e9, "frac": nbytes / med / 1e9 / peak}
         pool.close()
     torch.cuda.empty_cache()
+    return out
+
+
+def gdn_pivot_heads(stq, flush, stream, peak, R: int = 64, pivots: int = 11, reps: int = 20):
+    """The serving pool (R requests x 5 slots x 768 heads, mixed 6-bit GDN) with
+    `pivots` heads held in FP16 (the page keeps 32 of 2304 GDN heads so: 11 of 768),
+    one token per step over all heads (the fused kernel, then the pivot heads'
+    kernel); median over `reps` steps with the L2 flushed before each, against the
+    same pool without pivot heads."""
+    import dataclasses
+    import torch
+    wl = synth.make_workload(4, R=R)
+    piv = wl.unit_bits.copy()
+    piv[np.linspace(0, wl.H - 1, pivots).astype(int)] = 16
+    req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
+    slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
+    x = {k: torch.from_numpy(v).cuda() for k, v in wl.step_inputs(0).items()}
+    y = torch.empty((wl.R, wl.H, 128), dtype=torch.float32, device="cuda")
+    out = {"requests": R, "slots": wl.S, "heads": wl.H, "pivot_heads": pivots}
+    for tag, bits in (("without", wl.unit_bits), ("with", piv)):
+        w = dataclasses.replace(wl, unit_bits=bits)
+        pool = stq.stq_pool_create(w.kind, w.R, w.S, w.H, bits, w.row_factor, w.col_factor)
+        S0 = w.initial_state()
+        if S0 is not None:
+            stq.stq_quantize_state(pool, req, slot, torch.from_numpy(S0).cuda())
+            del S0
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            stq.stq_decode_step(pool, req, slot, x["q"], x["k"], x["v"], x["beta"], x["gate"], y, stream)
+            b.record(stream)
+            if i >= 3:
+                ts.append((a, b))
+        torch.cuda.synchronize()
+        stq.stq_pool_check(pool, stream)
+        med = statistics.median(a.elapsed_time(b) for a, b in ts) * 1e-3
+        nbytes, _ = workload_info(w)
+        out[tag] = {"step_us": med * 1e6, "head_steps_per_s": R * wl.H / med, "gbs": nbytes / med / 1e9,
+                    "frac": nbytes / med / 1e9 / peak}
+        pool.close()
+        torch.cuda.empty_cache()
     return out
 
 

@@ -21,6 +21,7 @@ struct stq_pool {
     int scale_bytes = 4, raw_bits = 0;
     bool pivots = false;       // FP16 pivot units among quantized ones
     bool pivot_heads = false;  // GDN pivot heads (their own kernel)
+    int n_pivot_heads = 0;
     bool fit = false;          // per-page column factors refitted at every quantisation
     bool per_row = false;      // KDA: every tile on the decode kernel's per-row path
     int device = 0;
@@ -192,6 +193,7 @@ stq::PoolView view(stq_pool *p)
     v.pivots = p->pivots ? 1 : 0;
     v.fit = p->fit ? 1 : 0;
     v.per_row = p->per_row ? 1 : 0;
+    v.n_pivot_heads = p->n_pivot_heads;
     v.t = p->t;
     v.err = p->d_err;
     // STQ_FAULT=timeout: a wait that nothing completes, given a short limit
@@ -369,10 +371,11 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     const size_t n_hoff = (size_t)H * 4, n_pb = (size_t)H * 4, n_ro = (size_t)H * kD * 2,
                  n_rb = (size_t)H * kD, n_f = (size_t)H * kD * 4;
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t n_blk = (size_t)H * stq::kHeadBlock;
+    const size_t n_blk = (size_t)H * stq::kHeadBlock, n_ph = (size_t)H * 4;
     const size_t o_hoff = 0, o_pb = o_hoff + al(n_hoff), o_ro = o_pb + al(n_pb),
                  o_rb = o_ro + al(n_ro), o_r = o_rb + al(n_rb), o_c = o_r + al(n_f),
-                 o_w = o_c + al(n_f), o_blk = o_w + al(n_f), total = o_blk + al(n_blk);
+                 o_w = o_c + al(n_f), o_blk = o_w + al(n_f), o_ph = o_blk + al(n_blk),
+                 total = o_ph + al(n_ph);
     std::vector<uint8_t> img(total, 0);
     std::memcpy(&img[o_hoff], p->head_off.data(), n_hoff);
     std::memcpy(&img[o_pb], p->page_bytes.data(), n_pb);
@@ -381,6 +384,12 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
         std::memcpy(&img[o_ro + (size_t)h * kD * 2], L.row_off, kD * 2);
     }
     std::memcpy(&img[o_rb], rb.data(), n_rb);
+    if (p->pivot_heads) {
+        // the GDN pivot heads (every row at 16 bits), so that their kernel launches only their tiles
+        int32_t *ph = reinterpret_cast<int32_t *>(&img[o_ph]);
+        for (int h = 0; h < H; ++h)
+            if (rb[(size_t)h * kD] == 16) ph[p->n_pivot_heads++] = h;
+    }
     float *fr = reinterpret_cast<float *>(&img[o_r]);
     float *fc = reinterpret_cast<float *>(&img[o_c]);
     float *fw = reinterpret_cast<float *>(&img[o_w]);  // w_i, the column fit's row weights (1 without)
@@ -474,6 +483,7 @@ stq_status stq_pool_create(const stq_pool_desc *desc, stq_pool **out)
     p->t.c = reinterpret_cast<const float *>(base + o_c);
     p->t.w = reinterpret_cast<const float *>(base + o_w);
     p->t.block = base + o_blk;
+    p->t.pivot_head = reinterpret_cast<const int32_t *>(base + o_ph);
     *out = p;
     return STQ_OK;
 }

@@ -115,8 +115,16 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
     __shared__ float kqp[4];
     __shared__ uint32_t bad;
 
-    const int tile = blockIdx.x;
-    const int ni = tile / p.H, h = tile - ni * p.H;
+    // raw pools: block = tile; pivot heads: block = (entry, k-th pivot head)
+    int ni, h;
+    if (PIVOT) {
+        ni = blockIdx.x / p.n_pivot_heads;
+        h = p.t.pivot_head[blockIdx.x - ni * p.n_pivot_heads];
+    } else {
+        ni = blockIdx.x / p.H;
+        h = blockIdx.x - ni * p.H;
+    }
+    const int tile = ni * p.H + h;
     if (PIVOT && p.t.row_bits[h * kD] != 16) return;  // a quantized head: the fused kernel's
     const int req = io.req_idx[ni], slot = io.slot_idx[ni];
     const int tid = threadIdx.x;
@@ -231,7 +239,9 @@ __global__ void __launch_bounds__(kRawThreads, 2) decode_raw_kernel(PoolView p, 
 template <int KIND, int BITS, bool PIVOT = false>
 cudaError_t launch_raw(const PoolView &p, const DecodeIO &io, cudaStream_t stream)
 {
-    decode_raw_kernel<KIND, BITS, PIVOT><<<io.n * p.H, kRawThreads, 0, stream>>>(p, io);
+    const int blocks = io.n * (PIVOT ? p.n_pivot_heads : p.H);
+    if (blocks == 0) return cudaSuccess;
+    decode_raw_kernel<KIND, BITS, PIVOT><<<blocks, kRawThreads, 0, stream>>>(p, io);
     count_launch();
     return cudaGetLastError();
 }

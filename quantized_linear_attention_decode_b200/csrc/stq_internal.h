@@ -43,6 +43,7 @@ struct Tables {
     const float *c;
     const float *w;
     const uint8_t *block;
+    const int32_t *pivot_head;  // GDN: the FP16 pivot heads, ascending (n_pivot_heads of them)
 };
 
 struct PoolView {
@@ -56,6 +57,7 @@ struct PoolView {
     int fit;             // nonzero: pages carry column factors refitted at every quantisation
     int per_row;         // KDA: some head has a pass warp whose 16 rows the width-specialised
                          // passes cannot take, so every tile takes the per-row path
+    int n_pivot_heads;   // GDN: heads held in FP16 (their own kernel), listed in t.pivot_head
     Tables t;
     uint32_t *err;
     unsigned long long wait_ns;  // limit of every bounded device-side wait
