@@ -8,10 +8,12 @@
 //   y  = X^T q (before requantisation)   codes, scales = quantize_rows(X)
 //
 // Design (B200): persistent CTAs, two per SM, 256 threads each.  A CTA walks
-// its tiles (one (request, head) state each) in a fixed stride; thread 0
+// its tiles (one (request, head) state each) in a fixed stride; thread 96
 // keeps a four-stage ring of shared-memory buffers filled three tiles ahead
-// with bulk async copies (packed page, q, k, v, r, c, row tables, KDA decay),
-// completion tracked by one mbarrier per stage.  The requantised codes and
+// with bulk async copies (the packed page and the head's table block: r, c,
+// row offsets, widths and order), completion tracked by one mbarrier per
+// stage; q, k, v (and the KDA decay), beta and alpha come in by cp.async,
+// also three tiles ahead.  The requantised codes and
 // scales go from registers straight to the page in global memory (coalesced
 // per row).  Thread (rg, cg) owns rows [8 rg, 8 rg + 8)
 // and columns [8 cg, 8 cg + 8) of the 128 x 128 tile in registers as
@@ -22,7 +24,8 @@
 // Codes become floats with the 2^23 trick (a byte or field OR-ed into the
 // mantissa of 2^23, then 2^23 + 2^(b-1) subtracted), pairs of columns are
 // processed with packed fma.rn.f32x2, and requantised codes are read back
-// from the mantissa of fma(w, inv, 2^23 + 2^(b-1)).
+// from the mantissa of fma(w, inv, M_b) (M_b = 2^23 + 2^(b-1) at 4 and 6
+// bits, 1.5 * 2^23 at 8 bits).
 //
 // The same kernel, instantiated per mode, also runs the step split in two
 // ("method steps", steps 3-7: the readout first, the requantisation and
