@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=8)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--kda-allocated", action="store_true",
+                    help="config 3 with per-row widths from the allocator and 8 FP16 pivot rows per head "
+                         "(no CPU baseline, no recorded traffic)")
     ap.add_argument("--config", type=int, default=2, choices=[2, 3, 4],
                     help="2: GDN mixed 64 x 32 (default); 3: KDA 128 x 32; 4: serving pool (see --requests)")
     ap.add_argument("--requests", type=int, default=None, help="requests of the workload (default: its own)")
@@ -329,6 +332,12 @@ def run_ours(args, rank: int, world: int):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", dev))
     wl = synth.make_workload(args.config, seed=shard_seed(args.seed, rank), R=args.requests)
+    if args.kda_allocated:
+        if args.config != 3:
+            raise SystemExit("--kda-allocated needs --config 3")
+        import dataclasses
+        wl = dataclasses.replace(wl, unit_bits=kda_allocated_bits(stq, wl.H, 0),
+                                 name=wl.name.replace("mixed6", "allocated_pivots"))
     pool = stq.stq_pool_create(wl.kind, wl.R, wl.S, wl.H, wl.unit_bits, wl.row_factor, wl.col_factor)
     req = torch.arange(wl.R, dtype=torch.int32, device="cuda")
     slot = torch.from_numpy(wl.slot_of_request.astype(np.int32)).cuda()
@@ -383,7 +392,7 @@ def run_ours(args, rank: int, world: int):
     kernel_s = statistics.mean(times) * 1e-3
     peak, peak_kind = peaks()
     achieved = bytes_per_launch / kernel_s / 1e9
-    traffic = recorded_traffic(args.config, wl.R)
+    traffic = None if args.kda_allocated else recorded_traffic(args.config, wl.R)
 
     # ---- end to end through the public API: one pinned host block of inputs in,
     # y out, through stq_decode_step_host_block (its input copy and the decode,
@@ -458,7 +467,7 @@ def run_ours(args, rank: int, world: int):
             drift_log = drift(stq)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.kda_allocated:
         v, threads, sample, v1 = oracle_baseline(args.config, args.seed, args.cpu_seconds)
         cpu = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample,
                "value_1core": v1}
